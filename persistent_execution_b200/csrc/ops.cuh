@@ -1,0 +1,580 @@
+// ops.cuh -- op bodies: one work item of one op, run by a group of warps.
+//
+// The same bodies serve the persistent kernel (its compute warps) and the
+// one-kernel-per-op baseline, so both paths compute identical results. A body
+// sees the op's ring entry in shared memory, the item index, and a compute
+// context (thread index within the group, group size, a named barrier and a
+// small shared scratch). Elementwise items stream 16-byte vectors with several
+// loads in flight per thread; row items give each warp a row segment, reduce
+// with warp shuffles and combine segments through shared memory.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace gpuos_impl {
+
+struct Cx {
+  int tid, nthr;       // thread index in the compute group, group size
+  int warp, nwarps, lane;
+  int bar;             // named barrier id of the compute group
+  float4* part;        // shared scratch, >= nwarps entries
+};
+
+struct OpEnv {
+  DevState* st;        // null in the one-kernel-per-op baseline
+  HostCtl* hctl;
+  u64 timeout_ns;
+  u64 id;
+};
+
+__device__ __forceinline__ void cx_sync(const Cx& c) { bar_sync(c.bar, c.nthr); }
+
+// First device error wins; it is mirrored to the host control block, then the
+// abort flag tells every CTA to leave.
+static __device__ __noinline__ void raise_error(DevState* st, HostCtl* hctl, unsigned code, u64 id) {
+  if (st == nullptr) return;
+  u64 word = (u64)code | ((id + 1) << 8);
+  u64 old = atomicCAS(&st->err.v, 0ull, word);
+  if (old == 0) {
+    hctl->err_id = id;
+    fence_acq_rel_sys();
+    st_relaxed_sys32(&hctl->status, code);
+  }
+  st_release_gpu(&st->abort_.v, 1ull);
+}
+
+// ------------------------------------------------------------------ elements
+__device__ __forceinline__ float bf2f(unsigned short h) { return __uint_as_float((unsigned)h << 16); }
+__device__ __forceinline__ unsigned short f2bf(float f) { return __bfloat16_as_ushort(__float2bfloat16_rn(f)); }
+__device__ __forceinline__ bool al16(u64 p) { return (p & 15ull) == 0; }
+
+// 8 consecutive elements starting at element i (i % 8 == 0, base 16-byte aligned)
+template <int DT>
+__device__ __forceinline__ void ld8(u64 base, long long i, float (&v)[8]) {
+  if (DT == 0) {
+    const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + i);
+    float4 a = __ldcg(p), b = __ldcg(p + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+    uint4 r = __ldcg(reinterpret_cast<const uint4*>(reinterpret_cast<const unsigned short*>(base) + i));
+    unsigned w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[2 * j] = __uint_as_float(w[j] << 16);
+      v[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+    }
+  }
+}
+template <int DT>
+__device__ __forceinline__ void st8(u64 base, long long i, const float (&v)[8]) {
+  if (DT == 0) {
+    float4* p = reinterpret_cast<float4*>(reinterpret_cast<float*>(base) + i);
+    p[0] = make_float4(v[0], v[1], v[2], v[3]);
+    p[1] = make_float4(v[4], v[5], v[6], v[7]);
+  } else {
+    uint4 r;
+    r.x = (unsigned)f2bf(v[0]) | ((unsigned)f2bf(v[1]) << 16);
+    r.y = (unsigned)f2bf(v[2]) | ((unsigned)f2bf(v[3]) << 16);
+    r.z = (unsigned)f2bf(v[4]) | ((unsigned)f2bf(v[5]) << 16);
+    r.w = (unsigned)f2bf(v[6]) | ((unsigned)f2bf(v[7]) << 16);
+    *reinterpret_cast<uint4*>(reinterpret_cast<unsigned short*>(base) + i) = r;
+  }
+}
+template <int DT>
+__device__ __forceinline__ float ld1(u64 base, long long i) {
+  if (DT == 0) return __ldcg(reinterpret_cast<const float*>(base) + i);
+  return bf2f(__ldcg(reinterpret_cast<const unsigned short*>(base) + i));
+}
+template <int DT>
+__device__ __forceinline__ void st1(u64 base, long long i, float v) {
+  if (DT == 0)
+    reinterpret_cast<float*>(base)[i] = v;
+  else
+    reinterpret_cast<unsigned short*>(base)[i] = f2bf(v);
+}
+
+// ------------------------------------------------------------------ scalar defs
+__device__ __forceinline__ float relu_f(float v) { return (v <= 0.0f) ? 0.0f : v; }  // NaN passes, -0 -> +0
+// The double-precision transcendentals stay out of line: inlined into the
+// unrolled vector loops they would multiply register pressure for every op.
+static __device__ __noinline__ float gelu_f(float x) {
+  double xd = (double)x;
+  return (float)(0.5 * xd * erfc(-xd / 1.4142135623730951));
+}
+static __device__ __noinline__ float silu_f(float x) {
+  double xd = (double)x;
+  return (float)(xd / (1.0 + exp(-xd)));
+}
+static __device__ __noinline__ float silu_mul_f(float g, float u) {
+  double gd = (double)g;
+  return (float)(gd / (1.0 + exp(-gd)) * (double)u);
+}
+
+// Fused micro-op program over one element; the program and scalars are read
+// from the shared-memory entry (uniform across the group).
+__device__ __forceinline__ float chain_f(const RingEntry& E, float acc, float x1, float x2) {
+  int k = 0;
+  const int nm = E.nmicro;
+  for (int i = 0; i < nm; ++i) {
+    switch (E.micro[i]) {
+      case GPUOS_M_AFFINE: acc = __fmaf_rn(E.s[k & 3], acc, E.s[(k + 1) & 3]); k += 2; break;
+      case GPUOS_M_SCALE: acc = __fmul_rn(acc, E.s[k & 3]); k += 1; break;
+      case GPUOS_M_ADDS: acc = __fadd_rn(acc, E.s[k & 3]); k += 1; break;
+      case GPUOS_M_RELU: acc = relu_f(acc); break;
+      case GPUOS_M_GELU: acc = gelu_f(acc); break;
+      case GPUOS_M_SILU: acc = silu_f(acc); break;
+      case GPUOS_M_ADD1: acc = __fadd_rn(acc, x1); break;
+      case GPUOS_M_MUL1: acc = __fmul_rn(acc, x1); break;
+      case GPUOS_M_ADD2: acc = __fadd_rn(acc, x2); break;
+      case GPUOS_M_MUL2: acc = __fmul_rn(acc, x2); break;
+      default: break;
+    }
+  }
+  return acc;
+}
+
+template <int OPK>
+__device__ __forceinline__ float ew_f(const RingEntry& E, float x0, float x1, float x2) {
+  if (OPK == GPUOS_OP_ADD) return __fadd_rn(x0, x1);
+  if (OPK == GPUOS_OP_MUL) return __fmul_rn(x0, x1);
+  if (OPK == GPUOS_OP_SCALE) return __fmul_rn(E.s[0], x0);
+  if (OPK == GPUOS_OP_GELU) return gelu_f(x0);
+  if (OPK == GPUOS_OP_RELU_AFFINE) return relu_f(__fmaf_rn(E.s[0], x0, E.s[1]));
+  if (OPK == GPUOS_OP_SILU_MUL) return silu_mul_f(x0, x1);
+  return chain_f(E, x0, x1, x2);  // GPUOS_OP_EW_CHAIN, OPK_CHAIN_CALLS
+}
+
+// Program-wide micro-op loop for one vector of 8 elements: the micro-op
+// switch is taken once per vector instead of once per element.
+__device__ __forceinline__ void chain8(const RingEntry& E, float (&a)[8], const float (&x1)[8],
+                                       const float (&x2)[8]) {
+  int k = 0;
+  const int nm = E.nmicro;
+  for (int i = 0; i < nm; ++i) {
+    const int m = E.micro[i];
+    if (m == GPUOS_M_AFFINE) {
+      const float s0 = E.s[k & 3], s1 = E.s[(k + 1) & 3];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a[j] = __fmaf_rn(s0, a[j], s1);
+      k += 2;
+    } else if (m == GPUOS_M_RELU) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a[j] = relu_f(a[j]);
+    } else if (m == GPUOS_M_SCALE) {
+      const float s0 = E.s[k & 3];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a[j] = __fmul_rn(a[j], s0);
+      k += 1;
+    } else if (m == GPUOS_M_ADDS) {
+      const float s0 = E.s[k & 3];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a[j] = __fadd_rn(a[j], s0);
+      k += 1;
+    } else if (m == GPUOS_M_ADD1) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a[j] = __fadd_rn(a[j], x1[j]);
+    } else if (m == GPUOS_M_MUL1) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a[j] = __fmul_rn(a[j], x1[j]);
+    } else if (m == GPUOS_M_ADD2) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a[j] = __fadd_rn(a[j], x2[j]);
+    } else if (m == GPUOS_M_MUL2) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a[j] = __fmul_rn(a[j], x2[j]);
+    }
+  }
+}
+
+__device__ __forceinline__ void chain_uses(const RingEntry& E, bool& u1, bool& u2) {
+  u1 = u2 = false;
+  for (int i = 0; i < E.nmicro; ++i) {
+    const int m = E.micro[i];
+    u1 |= (m == GPUOS_M_ADD1 || m == GPUOS_M_MUL1);
+    u2 |= (m == GPUOS_M_ADD2 || m == GPUOS_M_MUL2);
+  }
+}
+
+constexpr int EW_UNR = 4;  // vectors of 8 elements in flight per thread
+
+// Pseudo-opcode: a fused program that calls an out-of-line transcendental
+// (gelu, silu) runs element by element, without the unrolled vector batch.
+constexpr int OPK_CHAIN_CALLS = 1000;
+
+// Each body is out of line: inlined together into one dispatcher, the union
+// of their unrolled register arrays would spill.
+template <int DT, int OPK, int UNR>
+static __device__ __noinline__ void ew_loop(const RingEntry& E, u32 item, u32 elem_chunk, const Cx cx) {
+  const long long n = E.rows * E.cols;
+  const long long e0 = (long long)item * elem_chunk;
+  const long long e1 = min(n, e0 + (long long)elem_chunk);
+  bool u1, u2;
+  if (OPK == GPUOS_OP_EW_CHAIN || OPK == OPK_CHAIN_CALLS) {
+    chain_uses(E, u1, u2);
+  } else {
+    u1 = (OPK == GPUOS_OP_ADD || OPK == GPUOS_OP_MUL || OPK == GPUOS_OP_SILU_MUL);
+    u2 = false;
+  }
+  const long long n0 = E.in_n0, n1 = E.in_n1;
+  const bool vec = al16(E.in0) && al16(E.out) && n0 == n && (!u1 || (n1 == n && al16(E.in1))) &&
+                   (!u2 || al16(E.in2));
+  if (vec) {
+    const long long v0 = e0 >> 3, v1 = e1 >> 3;  // whole vectors of this item
+    for (long long v = v0 + cx.tid; v < v1; v += (long long)UNR * cx.nthr) {
+      float a[UNR][8], b[UNR][8], c[UNR][8];
+#pragma unroll
+      for (int u = 0; u < UNR; ++u) {
+        const long long vi = v + (long long)u * cx.nthr;
+        if (vi < v1) {
+          ld8<DT>(E.in0, vi << 3, a[u]);
+          if (u1) ld8<DT>(E.in1, vi << 3, b[u]);
+          else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) b[u][j] = 0.f;
+          }
+          if (u2) ld8<DT>(E.in2, vi << 3, c[u]);
+          else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) c[u][j] = 0.f;
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < UNR; ++u) {
+        const long long vi = v + (long long)u * cx.nthr;
+        if (vi < v1) {
+          if (OPK == GPUOS_OP_EW_CHAIN) {
+            chain8(E, a[u], b[u], c[u]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) a[u][j] = ew_f<OPK>(E, a[u][j], b[u][j], c[u][j]);
+          }
+          st8<DT>(E.out, vi << 3, a[u]);
+        }
+      }
+    }
+    for (long long e = (v1 << 3) + cx.tid; e < e1; e += cx.nthr) {  // ragged tail (< 8 elements)
+      const float x0 = ld1<DT>(E.in0, e);
+      const float x1 = u1 ? ld1<DT>(E.in1, e) : 0.f;
+      const float x2 = u2 ? ld1<DT>(E.in2, e) : 0.f;
+      st1<DT>(E.out, e, ew_f<OPK>(E, x0, x1, x2));
+    }
+  } else {
+    for (long long e = e0 + cx.tid; e < e1; e += cx.nthr) {
+      const float x0 = ld1<DT>(E.in0, n0 == n ? e : e % n0);
+      const float x1 = u1 ? ld1<DT>(E.in1, n1 == n ? e : e % n1) : 0.f;
+      const float x2 = u2 ? ld1<DT>(E.in2, e) : 0.f;
+      st1<DT>(E.out, e, ew_f<OPK>(E, x0, x1, x2));
+    }
+  }
+}
+
+__device__ __forceinline__ bool chain_calls(const RingEntry& E) {
+  bool c = false;
+  for (int i = 0; i < E.nmicro; ++i) c |= (E.micro[i] == GPUOS_M_GELU || E.micro[i] == GPUOS_M_SILU);
+  return c;
+}
+
+template <int DT>
+__device__ void ew_item(const RingEntry& E, u32 item, u32 elem_chunk, const Cx& cx) {
+  switch (E.opcode) {
+    case GPUOS_OP_ADD: ew_loop<DT, GPUOS_OP_ADD, EW_UNR>(E, item, elem_chunk, cx); break;
+    case GPUOS_OP_MUL: ew_loop<DT, GPUOS_OP_MUL, EW_UNR>(E, item, elem_chunk, cx); break;
+    case GPUOS_OP_SCALE: ew_loop<DT, GPUOS_OP_SCALE, EW_UNR>(E, item, elem_chunk, cx); break;
+    case GPUOS_OP_GELU: ew_loop<DT, GPUOS_OP_GELU, 1>(E, item, elem_chunk, cx); break;
+    case GPUOS_OP_RELU_AFFINE: ew_loop<DT, GPUOS_OP_RELU_AFFINE, EW_UNR>(E, item, elem_chunk, cx); break;
+    case GPUOS_OP_SILU_MUL: ew_loop<DT, GPUOS_OP_SILU_MUL, 1>(E, item, elem_chunk, cx); break;
+    default:
+      if (chain_calls(E))
+        ew_loop<DT, OPK_CHAIN_CALLS, 1>(E, item, elem_chunk, cx);
+      else
+        ew_loop<DT, GPUOS_OP_EW_CHAIN, EW_UNR>(E, item, elem_chunk, cx);
+      break;
+  }
+}
+
+// ------------------------------------------------------------------ row ops
+struct Acc {
+  float a, b;
+};
+
+__device__ __forceinline__ Acc acc_init(int op) {
+  if (op == GPUOS_OP_ROWMAX || op == GPUOS_OP_SOFTMAX) return Acc{-INFINITY, 0.f};
+  return Acc{0.f, 0.f};
+}
+
+// Folds 8 elements into a partial row statistic.
+__device__ __forceinline__ void acc8(int op, Acc& A, const float (&x)[8], float K) {
+  if (op == GPUOS_OP_ROWSUM) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) A.a += x[j];
+  } else if (op == GPUOS_OP_ROWMAX) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) A.a = fmaxf(A.a, x[j]);
+  } else if (op == GPUOS_OP_SOFTMAX) {
+    float m = A.a;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m = fmaxf(m, x[j]);
+    float s = (A.a == -INFINITY) ? 0.f : A.b * expf(A.a - m);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) s += expf(x[j] - m);
+    A.a = m;
+    A.b = s;
+  } else if (op == GPUOS_OP_RMSNORM) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) A.a = __fmaf_rn(x[j], x[j], A.a);
+  } else {  // LAYERNORM: shifted sums
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float d = x[j] - K;
+      A.a += d;
+      A.b = __fmaf_rn(d, d, A.b);
+    }
+  }
+}
+__device__ __forceinline__ void acc1(int op, Acc& A, float x, float K) {
+  if (op == GPUOS_OP_ROWSUM) {
+    A.a += x;
+  } else if (op == GPUOS_OP_ROWMAX) {
+    A.a = fmaxf(A.a, x);
+  } else if (op == GPUOS_OP_SOFTMAX) {
+    const float m = fmaxf(A.a, x);
+    A.b = ((A.a == -INFINITY) ? 0.f : A.b * expf(A.a - m)) + expf(x - m);
+    A.a = m;
+  } else if (op == GPUOS_OP_RMSNORM) {
+    A.a = __fmaf_rn(x, x, A.a);
+  } else {
+    const float d = x - K;
+    A.a += d;
+    A.b = __fmaf_rn(d, d, A.b);
+  }
+}
+__device__ __forceinline__ void acc_merge(int op, Acc& A, const Acc& B) {
+  if (op == GPUOS_OP_ROWMAX) {
+    A.a = fmaxf(A.a, B.a);
+  } else if (op == GPUOS_OP_SOFTMAX) {
+    const float m = fmaxf(A.a, B.a);
+    if (m != -INFINITY) {
+      A.b = A.b * expf(A.a - m) + B.b * expf(B.a - m);
+      A.a = m;
+    }
+  } else {
+    A.a += B.a;
+    A.b += B.b;
+  }
+}
+__device__ __forceinline__ void acc_warp(int op, Acc& A) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    Acc B{__shfl_xor_sync(0xffffffffu, A.a, off), __shfl_xor_sync(0xffffffffu, A.b, off)};
+    acc_merge(op, A, B);
+  }
+}
+
+// Writes the outputs of columns [c0, c1) of one row from its full statistic.
+template <int DT>
+__device__ void row_out(const RingEntry& E, int op, long long rb, long long c0, long long c1, Acc A, float K,
+                        bool vec, int lane) {
+  const long long cols = E.cols;
+  const float eps = E.s[0];
+  float p0 = 0.f, p1 = 0.f;  // per-row constants
+  if (op == GPUOS_OP_SOFTMAX) {
+    p0 = A.a;
+    p1 = A.b;
+  } else if (op == GPUOS_OP_RMSNORM) {
+    p0 = 1.0f / sqrtf(A.a / (float)cols + eps);
+  } else {  // LAYERNORM
+    const float mean_d = A.a / (float)cols;
+    float var = (A.b - A.a * mean_d) / (float)cols;
+    var = fmaxf(var, 0.f);
+    p0 = K + mean_d;
+    p1 = 1.0f / sqrtf(var + eps);
+  }
+  if (vec) {
+    for (long long c = c0 + (long long)lane * 8; c < c1; c += 256) {
+      float x[8], y[8];
+      ld8<DT>(E.in0, rb + c, x);
+      if (op == GPUOS_OP_SOFTMAX) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) y[j] = __fdiv_rn(expf(x[j] - p0), p1);
+      } else if (op == GPUOS_OP_RMSNORM) {
+        float w[8];
+        ld8<DT>(E.in1, c, w);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) y[j] = __fmul_rn(__fmul_rn(x[j], p0), w[j]);
+      } else {
+        float g[8], b[8];
+        ld8<DT>(E.in1, c, g);
+        ld8<DT>(E.in2, c, b);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) y[j] = __fmaf_rn(__fmul_rn(x[j] - p0, p1), g[j], b[j]);
+      }
+      st8<DT>(E.out, rb + c, y);
+    }
+  } else {
+    for (long long c = c0 + lane; c < c1; c += 32) {
+      const float x = ld1<DT>(E.in0, rb + c);
+      float y;
+      if (op == GPUOS_OP_SOFTMAX)
+        y = __fdiv_rn(expf(x - p0), p1);
+      else if (op == GPUOS_OP_RMSNORM)
+        y = __fmul_rn(__fmul_rn(x, p0), ld1<DT>(E.in1, c));
+      else
+        y = __fmaf_rn(__fmul_rn(x - p0, p1), ld1<DT>(E.in1, c), ld1<DT>(E.in2, c));
+      st1<DT>(E.out, rb + c, y);
+    }
+  }
+}
+
+constexpr int ROW_UNR = 4;
+
+// cos and sin of pos * base^(-2i/cols), in double.
+static __device__ __noinline__ double2 rotary_cs(double base, long long i, long long cols, int pos) {
+  const double theta = pow(base, (-2.0 * (double)i) / (double)cols);
+  const double phi = (double)pos * theta;
+  double sn, cs;
+  sincos(phi, &sn, &cs);
+  return make_double2(cs, sn);
+}
+
+template <int DT>
+static __device__ __noinline__ void rotary_item(const RingEntry& E, long long r0, int R, const Cx cx) {
+  const long long cols = E.cols, half = cols / 2;
+  const long long total = (long long)R * half;
+  const double base = (double)E.s[0];
+  for (long long p = cx.tid; p < total; p += cx.nthr) {
+    const long long row = p / half, i = p % half;
+    const double2 t = rotary_cs(base, i, cols, E.pos);
+    const double cs = t.x, sn = t.y;
+    const long long rb = (r0 + row) * cols;
+    const double x1 = (double)ld1<DT>(E.in0, rb + i), x2 = (double)ld1<DT>(E.in0, rb + i + half);
+    st1<DT>(E.out, rb + i, (float)(x1 * cs - x2 * sn));
+    st1<DT>(E.out, rb + i + half, (float)(x2 * cs + x1 * sn));
+  }
+}
+
+template <int DT>
+static __device__ __noinline__ void row_item(const RingEntry& E, u32 item, u32 row_chunk, const Cx cx) {
+  const long long rows = E.rows, cols = E.cols;
+  const long long rpi = rows_per_item(cols, row_chunk);
+  const long long r0 = (long long)item * rpi;
+  const int R = (int)min(rpi, rows - r0);
+  const int op = E.opcode;
+  if (op == GPUOS_OP_ROTARY) {
+    rotary_item<DT>(E, r0, R, cx);
+    return;
+  }
+  int S = 1;  // warps per row
+  while (2 * S * R <= cx.nwarps && cols / (2 * S) >= 256) S *= 2;
+  long long seg = (cols + S - 1) / S;
+  seg = (seg + 7) & ~7ll;
+  const int tasks = R * S;
+  bool vec = al16(E.in0) && (cols % 8) == 0;
+  if (op == GPUOS_OP_SOFTMAX || op == GPUOS_OP_RMSNORM || op == GPUOS_OP_LAYERNORM) vec = vec && al16(E.out);
+  if (op == GPUOS_OP_RMSNORM || op == GPUOS_OP_LAYERNORM) vec = vec && al16(E.in1);
+  if (op == GPUOS_OP_LAYERNORM) vec = vec && al16(E.in2);
+  const bool stats_only = (op == GPUOS_OP_ROWSUM || op == GPUOS_OP_ROWMAX);
+
+  for (int t = cx.warp; t < tasks; t += cx.nwarps) {
+    const int row = t / S, sg = t % S;
+    const long long c0 = (long long)sg * seg, c1 = min(cols, c0 + seg);
+    const long long rb = (r0 + row) * cols;
+    const float K = (op == GPUOS_OP_LAYERNORM) ? ld1<DT>(E.in0, rb) : 0.f;
+    Acc A = acc_init(op);
+    if (vec) {
+      long long c = c0 + (long long)cx.lane * 8;
+      for (; c + (long long)(ROW_UNR - 1) * 256 < c1; c += (long long)ROW_UNR * 256) {
+        float x[ROW_UNR][8];
+#pragma unroll
+        for (int u = 0; u < ROW_UNR; ++u) ld8<DT>(E.in0, rb + c + u * 256, x[u]);
+#pragma unroll
+        for (int u = 0; u < ROW_UNR; ++u) acc8(op, A, x[u], K);
+      }
+      for (; c < c1; c += 256) {
+        float x[8];
+        ld8<DT>(E.in0, rb + c, x);
+        acc8(op, A, x, K);
+      }
+    } else {
+      for (long long c = c0 + cx.lane; c < c1; c += 32) acc1(op, A, ld1<DT>(E.in0, rb + c), K);
+    }
+    acc_warp(op, A);
+    if (S == 1) {
+      if (stats_only) {
+        if (cx.lane == 0) st1<DT>(E.out, r0 + row, A.a);
+      } else {
+        row_out<DT>(E, op, rb, 0, cols, A, K, vec, cx.lane);
+      }
+    } else if (cx.lane == 0) {
+      cx.part[t] = make_float4(A.a, A.b, K, 0.f);
+    }
+  }
+  if (S > 1) {
+    cx_sync(cx);
+    for (int t = cx.warp; t < tasks; t += cx.nwarps) {
+      const int row = t / S, sg = t % S;
+      const long long c0 = (long long)sg * seg, c1 = min(cols, c0 + seg);
+      const long long rb = (r0 + row) * cols;
+      const float4 q0 = cx.part[row * S];
+      Acc A{q0.x, q0.y};
+      const float K = q0.z;
+      for (int j = 1; j < S; ++j) {
+        const float4 q = cx.part[row * S + j];
+        acc_merge(op, A, Acc{q.x, q.y});
+      }
+      if (stats_only) {
+        if (sg == 0 && cx.lane == 0) st1<DT>(E.out, r0 + row, A.a);
+      } else {
+        row_out<DT>(E, op, rb, c0, c1, A, K, vec, cx.lane);
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ dispatch
+__device__ __forceinline__ void stall_item(const OpEnv& env, const Cx& cx) {
+  if (cx.tid != 0 || env.st == nullptr) return;
+  const u64 t0 = globaltimer();
+  for (;;) {
+    if (ld_relaxed_sys(&env.hctl->stall_gate) != 0) break;
+    if (ld_relaxed_gpu(&env.st->abort_.v) != 0) break;
+    if (globaltimer() - t0 > env.timeout_ns) {
+      raise_error(env.st, env.hctl, GPUOS_ETIMEDOUT, env.id);
+      break;
+    }
+    __nanosleep(1000);
+  }
+}
+
+__device__ __forceinline__ void run_item(const RingEntry& E, u32 item, u32 elem_chunk, u32 row_chunk, const Cx& cx,
+                                         const OpEnv& env) {
+  const int op = E.opcode;
+  if (op == GPUOS_OP_NOP) return;
+  if (E.dtype <= 1) {
+    if (op_is_ew(op)) {
+      if (E.dtype == 0)
+        ew_item<0>(E, item, elem_chunk, cx);
+      else
+        ew_item<1>(E, item, elem_chunk, cx);
+      return;
+    }
+    if (op_is_row(op)) {
+      if (E.dtype == 0)
+        row_item<0>(E, item, row_chunk, cx);
+      else
+        row_item<1>(E, item, row_chunk, cx);
+      return;
+    }
+  }
+  if (op == GPUOS_OP_STALL) {
+    stall_item(env, cx);
+    return;
+  }
+  if (cx.tid == 0) raise_error(env.st, env.hctl, GPUOS_EBADOP, env.id);
+}
+
+}  // namespace gpuos_impl
