@@ -207,6 +207,26 @@ constexpr int OPK_CHAIN_CALLS = 1000;
 
 // Each body is out of line: inlined together into one dispatcher, the union
 // of their unrolled register arrays would spill.
+// e mod m, in 32 bits when both fit
+__device__ __forceinline__ u64 umod(u64 a, u64 m) {
+  if (((a | m) >> 32) == 0) return (u64)((u32)a % (u32)m);
+  return a % m;
+}
+
+// 8 elements e..e+7 of an operand of m elements read at index (e + t) mod m:
+// one modulo per block, eight independent loads in flight.
+template <int DT>
+__device__ __forceinline__ void gather8(u64 base, long long e, long long m, long long n, float (&v)[8]) {
+  long long j = (m == n) ? e : (long long)umod((u64)e, (u64)m);
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    v[t] = ld1<DT>(base, j);
+    j = (j + 1 == m) ? 0 : j + 1;
+  }
+}
+
+// Each body is out of line: inlined together into one dispatcher, the union
+// of their unrolled register arrays would spill.
 template <int DT, int OPK, int UNR>
 static __device__ __noinline__ void ew_loop(const RingEntry& E, u32 item, u32 elem_chunk, const Cx cx) {
   const long long n = E.rows * E.cols;
@@ -220,56 +240,68 @@ static __device__ __noinline__ void ew_loop(const RingEntry& E, u32 item, u32 el
     u2 = false;
   }
   const long long n0 = E.in_n0, n1 = E.in_n1;
-  const bool vec = al16(E.in0) && al16(E.out) && n0 == n && (!u1 || (n1 == n && al16(E.in1))) &&
-                   (!u2 || al16(E.in2));
-  if (vec) {
-    const long long v0 = e0 >> 3, v1 = e1 >> 3;  // whole vectors of this item
-    for (long long v = v0 + cx.tid; v < v1; v += (long long)UNR * cx.nthr) {
-      float a[UNR][8], b[UNR][8], c[UNR][8];
+  // per operand: direct 16-byte vectors, or 8-element gathers (broadcast or unaligned)
+  const bool v0d = n0 == n && al16(E.in0);
+  const bool v1d = !u1 || (n1 == n && al16(E.in1));
+  const bool v2d = !u2 || al16(E.in2);
+  const bool vout = al16(E.out);
+  const bool all_vec = v0d && v1d && v2d && vout;
+  const long long b0 = e0 >> 3, b1 = e1 >> 3;  // whole 8-element blocks of this item
+  for (long long v = b0 + cx.tid; v < b1; v += (long long)UNR * cx.nthr) {
+    float a[UNR][8], b[UNR][8], c[UNR][8];
 #pragma unroll
-      for (int u = 0; u < UNR; ++u) {
-        const long long vi = v + (long long)u * cx.nthr;
-        if (vi < v1) {
-          ld8<DT>(E.in0, vi << 3, a[u]);
-          if (u1) ld8<DT>(E.in1, vi << 3, b[u]);
-          else {
+    for (int u = 0; u < UNR; ++u) {
+      const long long vi = v + (long long)u * cx.nthr;
+      if (vi < b1) {
+        const long long e = vi << 3;
+        if (all_vec || v0d)
+          ld8<DT>(E.in0, e, a[u]);
+        else
+          gather8<DT>(E.in0, e, n0, n, a[u]);
+        if (u1) {
+          if (all_vec || (n1 == n && al16(E.in1)))
+            ld8<DT>(E.in1, e, b[u]);
+          else
+            gather8<DT>(E.in1, e, n1, n, b[u]);
+        } else {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) b[u][j] = 0.f;
-          }
-          if (u2) ld8<DT>(E.in2, vi << 3, c[u]);
-          else {
+          for (int j = 0; j < 8; ++j) b[u][j] = 0.f;
+        }
+        if (u2) {
+          if (all_vec || v2d)
+            ld8<DT>(E.in2, e, c[u]);
+          else
+            gather8<DT>(E.in2, e, n, n, c[u]);
+        } else {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) c[u][j] = 0.f;
-          }
+          for (int j = 0; j < 8; ++j) c[u][j] = 0.f;
         }
       }
+    }
 #pragma unroll
-      for (int u = 0; u < UNR; ++u) {
-        const long long vi = v + (long long)u * cx.nthr;
-        if (vi < v1) {
-          if (OPK == GPUOS_OP_EW_CHAIN) {
-            chain8(E, a[u], b[u], c[u]);
-          } else {
+    for (int u = 0; u < UNR; ++u) {
+      const long long vi = v + (long long)u * cx.nthr;
+      if (vi < b1) {
+        if (OPK == GPUOS_OP_EW_CHAIN) {
+          chain8(E, a[u], b[u], c[u]);
+        } else {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) a[u][j] = ew_f<OPK>(E, a[u][j], b[u][j], c[u][j]);
-          }
+          for (int j = 0; j < 8; ++j) a[u][j] = ew_f<OPK>(E, a[u][j], b[u][j], c[u][j]);
+        }
+        if (all_vec || vout) {
           st8<DT>(E.out, vi << 3, a[u]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) st1<DT>(E.out, (vi << 3) + j, a[u][j]);
         }
       }
     }
-    for (long long e = (v1 << 3) + cx.tid; e < e1; e += cx.nthr) {  // ragged tail (< 8 elements)
-      const float x0 = ld1<DT>(E.in0, e);
-      const float x1 = u1 ? ld1<DT>(E.in1, e) : 0.f;
-      const float x2 = u2 ? ld1<DT>(E.in2, e) : 0.f;
-      st1<DT>(E.out, e, ew_f<OPK>(E, x0, x1, x2));
-    }
-  } else {
-    for (long long e = e0 + cx.tid; e < e1; e += cx.nthr) {
-      const float x0 = ld1<DT>(E.in0, n0 == n ? e : e % n0);
-      const float x1 = u1 ? ld1<DT>(E.in1, n1 == n ? e : e % n1) : 0.f;
-      const float x2 = u2 ? ld1<DT>(E.in2, e) : 0.f;
-      st1<DT>(E.out, e, ew_f<OPK>(E, x0, x1, x2));
-    }
+  }
+  for (long long e = (b1 << 3) + cx.tid; e < e1; e += cx.nthr) {  // ragged tail (< 8 elements)
+    const float x0 = ld1<DT>(E.in0, n0 == n ? e : (long long)umod((u64)e, (u64)n0));
+    const float x1 = u1 ? ld1<DT>(E.in1, n1 == n ? e : (long long)umod((u64)e, (u64)n1)) : 0.f;
+    const float x2 = u2 ? ld1<DT>(E.in2, e) : 0.f;
+    st1<DT>(E.out, e, ew_f<OPK>(E, x0, x1, x2));
   }
 }
 

@@ -54,6 +54,7 @@ struct __align__(16) Slot {
 
 struct Smem {
   Slot slot[FIFO];
+  RingEntry stage[32];  // descriptors of the run claimed by try_extend
   u64 full_bar[FIFO];
   u64 done_bar[FIFO];
   u64 free_bar[FIFO];
@@ -71,6 +72,7 @@ struct Control {
   int lane;
   u64 k = 0;                      // items emitted
   u64 run_next = 0, run_end = 0;  // claimed run of FOLLOW ops
+  u64 run_first = 0;              // op of stage[0]
   u64 pending = 0;                // id + 1 of a large op waiting to open
   u64 pend_word = 0, pend_t = 0;  // progress watchdog of the pending open
   u64 dep_ok = 0;                 // id + 1 of the large op whose dependencies were seen
@@ -140,7 +142,9 @@ struct Control {
   __device__ __forceinline__ bool wait_deps(u64 id, u64 d0, u64 d1) { return wait_dep(d0, id) && wait_dep(d1, id); }
 
   // Copies one entry into the next FIFO slot and signals the compute warps.
-  __device__ __forceinline__ bool emit(u64 id, u32 item, u32 nitems, u32 claim) {
+  // The caller has read the entry's tag with acquire ordering (lane 0, or the
+  // staging lane); the warp barrier below orders every copying lane after it.
+  __device__ __forceinline__ bool emit(u64 id, u32 item, u32 nitems, u32 claim, const RingEntry* staged = nullptr) {
     const u32 slot = (u32)(k % FIFO);
     const u32 par = (u32)((k / FIFO) & 1) ^ 1u;
     u32 ok = 1;
@@ -156,10 +160,12 @@ struct Control {
     }
     if (bcast32(ok) == 0) return false;
     Slot& s = S->slot[slot];
+    __syncwarp();
     if (lane < 8) {
-      const RingEntry* src = ent(id);
-      (void)ld_acquire_gpu(&src->hdr);
-      reinterpret_cast<uint4*>(&s.e)[lane] = __ldcg(reinterpret_cast<const uint4*>(src) + lane);
+      if (staged)
+        reinterpret_cast<uint4*>(&s.e)[lane] = reinterpret_cast<const uint4*>(staged)[lane];
+      else
+        reinterpret_cast<uint4*>(&s.e)[lane] = __ldcg(reinterpret_cast<const uint4*>(ent(id)) + lane);
     }
     if (lane == 0) {
       s.id = id;
@@ -315,21 +321,34 @@ struct Control {
     u32 won = 0;
     if (lane == 0) won = atomicCAS(&p.st->next_op.v, c + 1, c + 1 + r) == c + 1;
     if (bcast32(won)) {
+      // each lane stages the descriptor whose tag it read with acquire ordering
+      if ((u32)lane < r) {
+        const uint4* src = reinterpret_cast<const uint4*>(ent(id));
+        uint4* dst = reinterpret_cast<uint4*>(&S->stage[lane]);
+        uint4 v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = __ldcg(src + j);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) dst[j] = v[j];
+      }
+      __syncwarp();
+      run_first = c + 1;
       run_next = c + 1;
       run_end = c + 1 + r;
     }
   }
 
-  __device__ __forceinline__ bool emit_single(u64 c, u32 claim) {
+  __device__ __forceinline__ bool emit_single(u64 c, u32 claim, const RingEntry* staged = nullptr) {
     u64 d0 = 0, d1 = 0;
     if (lane == 0) {
-      d0 = ent(c)->dep0;
-      d1 = ent(c)->dep1;
+      const RingEntry* e = staged ? staged : ent(c);
+      d0 = e->dep0;
+      d1 = e->dep1;
     }
     d0 = bcast(d0);
     d1 = bcast(d1);
     if (!wait_deps(c, d0, d1)) return false;
-    if (!emit(c, 0, 1, claim)) return false;
+    if (!emit(c, 0, 1, claim, staged)) return false;
     note_single(c);
     return true;
   }
@@ -480,7 +499,7 @@ struct Control {
       if ((++iters & 63) == 0 && aborted_b()) break;
       if (run_next < run_end) {
         const u64 c = run_next;
-        if (!emit_single(c, CLAIM_RUN)) break;
+        if (!emit_single(c, CLAIM_RUN, &S->stage[c - run_first])) break;
         ++runops;
         ++run_next;
         if (run_next == run_end) try_extend(c);
@@ -525,53 +544,89 @@ struct Control {
 };
 
 // ------------------------------------------------------------------ publisher (one lane)
+// Publishes every item the compute warps have finished, in batches: one
+// device-scope fence makes the batch's outputs visible before its completion
+// words, one system-scope fence before the host completion entries.
+__device__ __forceinline__ bool mbar_test(unsigned long long* bar, unsigned int parity) {
+  unsigned int ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ void publisher(const KParams& p, Smem* S) {
   const bool trace = (p.flags & KF_TRACE) != 0;
   u64 items = 0, smin = ~0ull, smax = 0;
   const u32 sm = smid();
-  for (u64 k = 0;; ++k) {
-    const u32 slot = (u32)(k % FIFO);
-    const u32 par = (u32)((k / FIFO) & 1);
-    while (!mbar_try_wait(&S->done_bar[slot], par)) {
+  bool leave = false;
+  for (u64 k = 0; !leave;) {
+    {
+      const u32 slot = (u32)(k % FIFO);
+      while (!mbar_try_wait(&S->done_bar[slot], (u32)((k / FIFO) & 1))) {
+      }
     }
-    const Slot& s = S->slot[slot];
-    if (s.kind == SLOT_EXIT) break;
-    const u64 id = s.id;
-    const u64 idx = id & p.mask;
+    u32 m = 1;  // finished slots k .. k+m-1
+    while (m < FIFO && mbar_test(&S->done_bar[(k + m) % FIFO], (u32)(((k + m) / FIFO) & 1))) ++m;
+    u32 last_mask = 0, nwork = 0;
     fence_acq_rel_gpu();
-    bool last = true;
-    if (s.nitems > 1) {
-      const u32 old = atom_add_acq_rel_gpu(&p.tiles_done[idx], 1u);
-      last = (old + 1 == s.nitems);
-      if (last) p.tiles_done[idx] = 0u;
-    }
-    if (s.t_start < smin) smin = s.t_start;
-    if (s.t_end > smax) smax = s.t_end;
-    if (trace) {
-      gpuos_trace_rec* tr = &p.trace[idx];
-      if (s.nitems == 1) {
-        tr->t_start = s.t_start;
-        tr->t_end = s.t_end;
-        tr->items = 1;
-      } else {
-        atomicMin(reinterpret_cast<unsigned long long*>(&tr->t_start), s.t_start);
-        atomicMax(reinterpret_cast<unsigned long long*>(&tr->t_end), s.t_end);
-        atomicAdd(&tr->items, 1u);
+    for (u32 j = 0; j < m; ++j) {
+      const Slot& s = S->slot[(k + j) % FIFO];
+      if (s.kind == SLOT_EXIT) {
+        leave = true;
+        break;
+      }
+      ++nwork;
+      const u64 id = s.id;
+      const u64 idx = id & p.mask;
+      bool last = true;
+      if (s.nitems > 1) {
+        const u32 old = atom_add_acq_rel_gpu(&p.tiles_done[idx], 1u);
+        last = (old + 1 == s.nitems);
+        if (last) p.tiles_done[idx] = 0u;
+      }
+      if (s.t_start < smin) smin = s.t_start;
+      if (s.t_end > smax) smax = s.t_end;
+      if (trace) {
+        gpuos_trace_rec* tr = &p.trace[idx];
+        if (s.nitems == 1) {
+          tr->t_start = s.t_start;
+          tr->t_end = s.t_end;
+          tr->items = 1;
+        } else {
+          atomicMin(reinterpret_cast<unsigned long long*>(&tr->t_start), s.t_start);
+          atomicMax(reinterpret_cast<unsigned long long*>(&tr->t_end), s.t_end);
+          atomicAdd(&tr->items, 1u);
+        }
+        if (last) {
+          tr->cta = blockIdx.x;
+          tr->smid = sm;
+          tr->claim = s.claim;
+          tr->id = id + 1;
+        }
       }
       if (last) {
-        tr->cta = blockIdx.x;
-        tr->smid = sm;
-        tr->claim = s.claim;
-        tr->id = id + 1;
+        st_release_gpu(&p.done[idx], id + 1);
+        last_mask |= 1u << j;
       }
     }
-    if (last) {
-      st_release_gpu(&p.done[idx], id + 1);
-      atomicAdd(&p.st->ops_done.v, 1ull);
-      st_release_sys(&p.hdone[idx], id + 1);
+    if (last_mask) {
+      atomicAdd(&p.st->ops_done.v, (u64)__popc(last_mask));
+      fence_acq_rel_sys();
+      for (u32 j = 0; j < nwork; ++j) {
+        if (last_mask & (1u << j)) {
+          const u64 id = S->slot[(k + j) % FIFO].id;
+          st_relaxed_sys_u64(&p.hdone[id & p.mask], id + 1);
+        }
+      }
     }
-    mbar_arrive(&S->free_bar[slot]);
-    ++items;
+    for (u32 j = 0; j < nwork; ++j) mbar_arrive(&S->free_bar[(k + j) % FIFO]);
+    items += nwork;
+    k += nwork;
   }
   if (items) {
     atomicMin(&p.st->span_start.v, smin);

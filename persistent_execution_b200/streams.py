@@ -29,12 +29,15 @@ class DeviceArenas:
             self.upload(fill_outputs)
 
     def upload(self, fill_outputs=None):
+        """Copies the input region; the output region starts as zeros, or as
+        `fill_outputs` (NaN makes an op that never ran visible)."""
         w = self.w
-        self.f32.copy_(torch.from_numpy(w.arena_f32))
-        self.bf16.copy_(torch.from_numpy(w.arena_bf16.view(np.int16)).view(torch.bfloat16))
-        if fill_outputs is not None:  # poison outputs so an op that never ran is visible
-            self.f32[w.n_init_f32:].fill_(fill_outputs)
-            self.bf16[w.n_init_bf16:].fill_(fill_outputs)
+        self.f32[:w.n_init_f32].copy_(torch.from_numpy(w.arena_f32[:w.n_init_f32]))
+        self.bf16[:w.n_init_bf16].copy_(
+            torch.from_numpy(w.arena_bf16[:w.n_init_bf16].view(np.int16)).view(torch.bfloat16))
+        fill = 0.0 if fill_outputs is None else fill_outputs
+        self.f32[w.n_init_f32:].fill_(fill)
+        self.bf16[w.n_init_bf16:].fill_(fill)
 
     def download(self):
         a32 = self.f32.cpu().numpy()

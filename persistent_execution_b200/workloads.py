@@ -231,7 +231,15 @@ def config2(n_ops: int = 20000, nmin: int = 256, nmax: int = 65536, seed: int = 
     deps = []
     for i in range(n_ops):
         k = min(int(ndeps[i]), i)
-        deps.append(sorted(rng.choice(i, size=k, replace=False).tolist()) if k else [])
+        if k == 0:
+            deps.append([])
+        elif k == 1:
+            deps.append([int(rng.integers(0, i))])
+        else:  # two distinct earlier ops, uniformly
+            d0 = int(rng.integers(0, i))
+            d1 = int(rng.integers(0, i - 1))
+            d1 = d1 + 1 if d1 >= d0 else d1
+            deps.append(sorted([d0, d1]))
     # fresh inputs first (arena inputs precede outputs)
     fresh = {}
     for i in range(n_ops):
@@ -339,7 +347,7 @@ def config3(steps: int = 100, layers: int = 32, hidden: int = 2048, heads: int =
 # --------------------------------------------------------------------------
 # Config 4: dynamic-shape micro-batched serving stream
 # --------------------------------------------------------------------------
-def config4(n_ops: int = 100000, streams: int = 64, pool_elems: int = 64 << 20,
+def config4(n_ops: int = 100000, streams: int = 64, pool_elems: int = 16 << 20,
             hidden: int = 1024, lmin: int = 128, lmax: int = 4096, bmax: int = 8,
             seed: int = 3) -> Workload:
     """Round-robin interleaving of `streams` request chains; op i belongs to
