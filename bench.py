@@ -223,6 +223,18 @@ def bench_gpu(args, rank, world, local):
     rt = G.Runtime(stream.cuda_stream, flags=G.CFG_NO_AUTOSTART, ring_capacity=cap,
                    timeout_ns=10_000_000_000, idle_exit_ns=30_000_000_000)
 
+    if args.only_step:  # one drained step and nothing else (the command profiled with ncu)
+        rt.submit_n(descs, dep_base=0)
+        rt.flush()
+        rt.start(drain=True)
+        G.check(rt.wait(G.ALL, 120.0), "wait")
+        G.check(rt.stop(120.0), "stop")
+        rt.destroy()
+        stream.synchronize()
+        if rank == 0:
+            print(json.dumps({"only_step": True, "config": args.config, "ops": n}))
+        return
+
     def step_loop(k, events=None):
         """k drained steps; the next step's ops are written while the kernel runs."""
         for i in range(k):
@@ -397,6 +409,8 @@ def main():
     ap.add_argument("--impl", default="persistent", choices=["persistent", "reference"])
     ap.add_argument("--baselines", type=int, default=1)
     ap.add_argument("--ref-sample", type=int, default=0)
+    ap.add_argument("--only-step", action="store_true",
+                    help="run one drained step of the stream and exit (for ncu captures)")
     args = ap.parse_args()
     rank, world, local = setup_dist(args)
     try:
