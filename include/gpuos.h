@@ -250,6 +250,31 @@ gpuos_status gpuos_graph_create(const gpuos_desc* descs, uint64_t n, uint64_t de
 gpuos_status gpuos_graph_launch(gpuos_graph_t* g, gpuos_stream_t stream);
 gpuos_status gpuos_graph_destroy(gpuos_graph_t* g);
 
+/* ---------------------------------------------------------------- allocation-free variant */
+
+/* The pages have no counterpart of this call; it exists for callers that must
+ * not allocate. cudaMalloc, cudaHostAlloc and cudaFree can stall the whole
+ * device for milliseconds and fail when another allocator (PyTorch's caching
+ * allocator, for example) already holds the memory, so a latency-critical
+ * caller, or one whose device memory belongs to someone else, cannot use
+ * gpuos_create. gpuos_run_static runs descs[0..n) as one drained session of
+ * the persistent kernel without allocating anything: the ring, completion
+ * words and scheduler state live in a fixed array of about 620 KB inside the
+ * library (every GPU that loads the library holds it until the process exits).
+ *   - n <= 4096 and no GPUOS_OP_STALL ops, else GPUOS_EINVAL; at most 256 CTAs.
+ *   - Dependencies are indices into descs (an index below the op's own).
+ *   - Tensors are caller-owned device memory, as for gpuos_submit.
+ *   - Synchronous: returns once every op completed (or a device error, which
+ *     is returned, not kept). Uses `stream` for its copies and launches.
+ *   - The first call on a device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - Every call uses the same array and leaves it as the last call left it
+ *     (each call clears what must start at zero). Calls that overlap on the
+ *     GPU -- from two host threads, or on two streams -- race and corrupt
+ *     each other's state. */
+gpuos_status gpuos_run_static(const gpuos_desc* descs, uint64_t n, const gpuos_config* cfg,
+                              gpuos_stream_t stream);
+
 /* ---------------------------------------------------------------- host-only helpers */
 
 /* Checks a descriptor as gpuos_submit does, without a runtime or GPU. */

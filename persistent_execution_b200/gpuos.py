@@ -98,6 +98,7 @@ _SIGS = {
     "gpuos_validate": [_vp],
     "gpuos_debug_submit_raw": [_vp, _vp, ctypes.POINTER(_u64)],
     "gpuos_debug_release_stall": [_vp],
+    "gpuos_run_static": [_vp, _u64, ctypes.POINTER(Config), _vp],
 }
 
 
@@ -215,6 +216,10 @@ def gpuos_debug_submit_raw(rt, desc: np.ndarray, id_out: ctypes.c_uint64 = None)
 
 def gpuos_debug_release_stall(rt) -> int:
     return lib().gpuos_debug_release_stall(rt)
+
+
+def gpuos_run_static(descs: np.ndarray, n: int, cfg: Config, stream: int) -> int:
+    return lib().gpuos_run_static(_ptr(descs), n, ctypes.byref(cfg) if cfg is not None else None, _vp(stream))
 
 
 # ---------------------------------------------------------------- convenience wrapper
