@@ -199,7 +199,7 @@ __device__ __forceinline__ void chain_uses(const RingEntry& E, bool& u1, bool& u
   }
 }
 
-constexpr int EW_UNR = 4;  // vectors of 8 elements in flight per thread
+constexpr int EW_UNR = 2;  // 8-element blocks in flight per thread (binary ops; unary ops use twice as many)
 
 // Pseudo-opcode: a fused program that calls an out-of-line transcendental
 // (gelu, silu) runs element by element, without the unrolled vector batch.
@@ -227,17 +227,19 @@ __device__ __forceinline__ void gather8(u64 base, long long e, long long m, long
 
 // Each body is out of line: inlined together into one dispatcher, the union
 // of their unrolled register arrays would spill.
-template <int DT, int OPK, int UNR>
+// CH: which extra operands the body reads (bit 0: in1, bit 1: in2), or -1 to
+// decide at run time from the fused program.
+template <int DT, int OPK, int UNR, int CH>
 static __device__ __noinline__ void ew_loop(const RingEntry& E, u32 item, u32 elem_chunk, const Cx cx) {
   const long long n = E.rows * E.cols;
   const long long e0 = (long long)item * elem_chunk;
   const long long e1 = min(n, e0 + (long long)elem_chunk);
   bool u1, u2;
-  if (OPK == GPUOS_OP_EW_CHAIN || OPK == OPK_CHAIN_CALLS) {
+  if (CH < 0) {
     chain_uses(E, u1, u2);
   } else {
-    u1 = (OPK == GPUOS_OP_ADD || OPK == GPUOS_OP_MUL || OPK == GPUOS_OP_SILU_MUL);
-    u2 = false;
+    u1 = (CH & 1) != 0;
+    u2 = (CH & 2) != 0;
   }
   const long long n0 = E.in_n0, n1 = E.in_n1;
   // per operand: direct 16-byte vectors, or 8-element gathers (broadcast or unaligned)
@@ -314,17 +316,28 @@ __device__ __forceinline__ bool chain_calls(const RingEntry& E) {
 template <int DT>
 __device__ void ew_item(const RingEntry& E, u32 item, u32 elem_chunk, const Cx& cx) {
   switch (E.opcode) {
-    case GPUOS_OP_ADD: ew_loop<DT, GPUOS_OP_ADD, EW_UNR>(E, item, elem_chunk, cx); break;
-    case GPUOS_OP_MUL: ew_loop<DT, GPUOS_OP_MUL, EW_UNR>(E, item, elem_chunk, cx); break;
-    case GPUOS_OP_SCALE: ew_loop<DT, GPUOS_OP_SCALE, EW_UNR>(E, item, elem_chunk, cx); break;
-    case GPUOS_OP_GELU: ew_loop<DT, GPUOS_OP_GELU, 1>(E, item, elem_chunk, cx); break;
-    case GPUOS_OP_RELU_AFFINE: ew_loop<DT, GPUOS_OP_RELU_AFFINE, EW_UNR>(E, item, elem_chunk, cx); break;
-    case GPUOS_OP_SILU_MUL: ew_loop<DT, GPUOS_OP_SILU_MUL, 1>(E, item, elem_chunk, cx); break;
+    case GPUOS_OP_ADD: ew_loop<DT, GPUOS_OP_ADD, EW_UNR, 1>(E, item, elem_chunk, cx); break;
+    case GPUOS_OP_MUL: ew_loop<DT, GPUOS_OP_MUL, EW_UNR, 1>(E, item, elem_chunk, cx); break;
+    case GPUOS_OP_SCALE: ew_loop<DT, GPUOS_OP_SCALE, 2 * EW_UNR, 0>(E, item, elem_chunk, cx); break;
+    case GPUOS_OP_GELU: ew_loop<DT, GPUOS_OP_GELU, 1, 0>(E, item, elem_chunk, cx); break;
+    case GPUOS_OP_RELU_AFFINE: ew_loop<DT, GPUOS_OP_RELU_AFFINE, 2 * EW_UNR, 0>(E, item, elem_chunk, cx); break;
+    case GPUOS_OP_SILU_MUL: ew_loop<DT, GPUOS_OP_SILU_MUL, 1, 1>(E, item, elem_chunk, cx); break;
     default:
-      if (chain_calls(E))
-        ew_loop<DT, OPK_CHAIN_CALLS, 1>(E, item, elem_chunk, cx);
-      else
-        ew_loop<DT, GPUOS_OP_EW_CHAIN, EW_UNR>(E, item, elem_chunk, cx);
+      if (chain_calls(E)) {
+        ew_loop<DT, OPK_CHAIN_CALLS, 1, -1>(E, item, elem_chunk, cx);
+      } else {
+        bool u1, u2;
+        chain_uses(E, u1, u2);
+        const int ch = (u1 ? 1 : 0) | (u2 ? 2 : 0);
+        if (ch == 0)
+          ew_loop<DT, GPUOS_OP_EW_CHAIN, 2 * EW_UNR, 0>(E, item, elem_chunk, cx);
+        else if (ch == 1)
+          ew_loop<DT, GPUOS_OP_EW_CHAIN, EW_UNR, 1>(E, item, elem_chunk, cx);
+        else if (ch == 2)
+          ew_loop<DT, GPUOS_OP_EW_CHAIN, EW_UNR, 2>(E, item, elem_chunk, cx);
+        else
+          ew_loop<DT, GPUOS_OP_EW_CHAIN, EW_UNR / 2, 3>(E, item, elem_chunk, cx);
+      }
       break;
   }
 }
@@ -462,7 +475,7 @@ __device__ void row_out(const RingEntry& E, int op, long long rb, long long c0, 
   }
 }
 
-constexpr int ROW_UNR = 4;
+constexpr int ROW_UNR = 8;
 
 // cos and sin of pos * base^(-2i/cols), in double.
 static __device__ __noinline__ double2 rotary_cs(double base, long long i, long long cols, int pos) {

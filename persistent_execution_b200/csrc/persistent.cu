@@ -38,6 +38,11 @@ namespace gpuos_impl {
 
 constexpr int NTHREADS = (NCW + 2) * 32;
 constexpr int FIFO = 8;
+// Items a CTA may have emitted but not finished before it claims another op
+// or joins a large op: a shallow window keeps ready ops from queueing behind
+// unrelated ones and keeps a large op's items from being hoarded long before
+// they run. Runs of FOLLOW ops use the whole FIFO.
+constexpr unsigned LOOKAHEAD = 2;
 constexpr unsigned FULLMASK = 0xffffffffu;
 
 enum : u32 { SLOT_WORK = 0, SLOT_EXIT = 1 };
@@ -60,6 +65,7 @@ struct Smem {
   u64 free_bar[FIFO];
   float4 part[NCW];
   u64 recent[8];
+  volatile unsigned ncomp;  // items the compute warps finished
 };
 
 __device__ __forceinline__ u64 bcast(u64 v) { return __shfl_sync(FULLMASK, v, 0); }
@@ -139,12 +145,50 @@ struct Control {
     return bcast32(ok) != 0;
   }
 
-  __device__ __forceinline__ bool wait_deps(u64 id, u64 d0, u64 d1) { return wait_dep(d0, id) && wait_dep(d1, id); }
+  // Both dependencies, polled together (one L2 round trip when both are done).
+  __device__ __forceinline__ bool wait_deps(u64 id, u64 d0, u64 d1) {
+    if (d0 != 0 && is_local(d0 - 1)) d0 = 0;
+    if (d1 != 0 && is_local(d1 - 1)) d1 = 0;
+    if (d0 == 0 || d1 == 0) return wait_dep(d0 | d1, id);
+    u32 ok = 0;
+    if (lane == 0) {
+      const u64 c0 = clock64();
+      const u64 t0 = globaltimer();
+      const u64* w0 = &p.done[(d0 - 1) & p.mask];
+      const u64* w1 = &p.done[(d1 - 1) & p.mask];
+      for (u32 spins = 0;; ++spins) {
+        const u64 v0 = ld_acquire_gpu(w0), v1 = ld_acquire_gpu(w1);
+        if (v0 >= d0 && v1 >= d1) {
+          ok = 1;
+          break;
+        }
+        if ((spins & 63) == 63) {
+          if (aborted()) break;
+          if (globaltimer() - t0 > p.timeout_ns) {
+            raise_error(p.st, p.hctl, GPUOS_ETIMEDOUT, id);
+            break;
+          }
+        }
+        if (spins > 64) __nanosleep(spins > 4096 ? 256 : 32);
+      }
+      dep_cyc += clock64() - c0;
+    }
+    return bcast32(ok) != 0;
+  }
+
+  // Waits until this CTA has fewer than `lim` items emitted but not finished.
+  __device__ __forceinline__ void throttle(unsigned lim) {
+    if (lane == 0) {
+      while ((unsigned)k - S->ncomp >= lim) __nanosleep(20);
+    }
+    __syncwarp();
+  }
 
   // Copies one entry into the next FIFO slot and signals the compute warps.
   // The caller has read the entry's tag with acquire ordering (lane 0, or the
   // staging lane); the warp barrier below orders every copying lane after it.
-  __device__ __forceinline__ bool emit(u64 id, u32 item, u32 nitems, u32 claim, const RingEntry* staged = nullptr) {
+  __device__ __forceinline__ bool emit(u64 id, u32 item, u32 nitems, u32 claim, const RingEntry* staged = nullptr,
+                                       bool have_reg = false, uint4 reg = uint4{0, 0, 0, 0}) {
     const u32 slot = (u32)(k % FIFO);
     const u32 par = (u32)((k / FIFO) & 1) ^ 1u;
     u32 ok = 1;
@@ -162,7 +206,9 @@ struct Control {
     Slot& s = S->slot[slot];
     __syncwarp();
     if (lane < 8) {
-      if (staged)
+      if (have_reg)
+        reinterpret_cast<uint4*>(&s.e)[lane] = reg;
+      else if (staged)
         reinterpret_cast<uint4*>(&s.e)[lane] = reinterpret_cast<const uint4*>(staged)[lane];
       else
         reinterpret_cast<uint4*>(&s.e)[lane] = __ldcg(reinterpret_cast<const uint4*>(ent(id)) + lane);
@@ -470,27 +516,47 @@ struct Control {
       if (lane == 0) ready = ld_acquire_gpu(&p.done[(c - 1) & p.mask]) >= c;
       if (!bcast32(ready)) return 0;  // the CTA that runs c - 1 is expected to take c
     }
+    // claim, and read the peeked entry in the same round trip (lane 0 read its
+    // tag with acquire ordering above; the warp barrier orders the other lanes)
+    __syncwarp();
     u64 c2 = 0;
+    uint4 chunk = uint4{0, 0, 0, 0};
     if (lane == 0) {
       if (hm - c > 2ull * p.grid + 64ull) {
         c2 = atomicAdd(&p.st->next_op.v, 1ull);
       } else {
         c2 = atomicCAS(&p.st->next_op.v, c, c + 1) == c ? c : ~0ull;
       }
-      if (c2 != ~0ull) st_relaxed_gpu(&p.st->activity.v, globaltimer());
     }
+    if (lane < 8) chunk = __ldcg(reinterpret_cast<const uint4*>(ent(c)) + lane);
+    if (lane == 0 && c2 != ~0ull) st_relaxed_gpu(&p.st->activity.v, globaltimer());
     c2 = bcast(c2);
     if (c2 == ~0ull) return 2;
     ++claimed;
     backoff = 0;
-    if (c2 != c && !wait_fetched(c2, h)) return -1;
+    if (c2 != c) {
+      if (!wait_fetched(c2, h)) return -1;
+      if (hdr_items(h) > 1) {
+        pending = c2 + 1;
+        pend_word = ~0ull;
+        return 1;
+      }
+      if (!emit_single(c2, CLAIM_SHARED)) return -1;
+      try_extend(c2);
+      return 1;
+    }
     if (hdr_items(h) > 1) {
       pending = c2 + 1;
       pend_word = ~0ull;
       return 1;
     }
-    if (!emit_single(c2, CLAIM_SHARED)) return -1;
-    try_extend(c2);
+    // dependencies straight from the entry in registers (dep0: lane 0, dep1: lane 1)
+    const u64 d0 = __shfl_sync(FULLMASK, (u64)chunk.z | ((u64)chunk.w << 32), 0);
+    const u64 d1 = __shfl_sync(FULLMASK, (u64)chunk.x | ((u64)chunk.y << 32), 1);
+    if (!wait_deps(c, d0, d1)) return -1;
+    if (!emit(c, 0, 1, CLAIM_SHARED, nullptr, true, chunk)) return -1;
+    note_single(c);
+    try_extend(c);
     return 1;
   }
 
@@ -506,6 +572,7 @@ struct Control {
         backoff = 0;
         continue;
       }
+      throttle(LOOKAHEAD);
       if (pending) {
         const int r = try_install(pending - 1);
         if (r < 0) break;
@@ -663,6 +730,7 @@ __device__ void compute(const KParams& p, Smem* S, int warp, int lane) {
     if (leader) {
       s.t_start = t0;
       s.t_end = globaltimer();
+      S->ncomp = (unsigned)(k + 1);
       mbar_arrive(&S->done_bar[slot]);
     }
   }
@@ -672,6 +740,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gpuos_persistent_kernel(const KPa
   __shared__ Smem S;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
+    S.ncomp = 0;
     for (int i = 0; i < FIFO; ++i) {
       mbar_init(&S.full_bar[i], 1);
       mbar_init(&S.done_bar[i], 1);
