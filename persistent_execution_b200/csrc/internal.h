@@ -2,6 +2,7 @@
 // persistent op-queue runtime (not part of the public ABI).
 #pragma once
 
+#include <cstddef>
 #include <cstdint>
 
 #include "../../include/gpuos.h"
@@ -149,6 +150,7 @@ struct KParams {
 int launch_session(const KParams& p, u64 head, u64 big_init, void* stream);
 int launch_op(const RingEntry& e, u32 elem_chunk, u32 row_chunk, u32 sms, void* stream);
 void* op_kernel_fn();
+size_t op_smem_bytes();
 void op_launch_dims(const RingEntry& e, u32 elem_chunk, u32 row_chunk, u32 sms, u32* grid, u32* block);
 
 }  // namespace gpuos_impl

@@ -16,11 +16,27 @@
 
 namespace gpuos_impl {
 
+// Shared-memory staging area of one compute warp: three stages, each armed
+// through its own mbarrier and filled by bulk asynchronous copies (the TMA
+// engine, no tensor map, no multicast).
+constexpr int WS_STAGES = 3;
+constexpr int WS_STAGE_BYTES = 4096;
+constexpr int WS_BYTES = WS_STAGES * WS_STAGE_BYTES;
+struct __align__(128) WarpSmem {
+  unsigned char buf[WS_BYTES];
+  unsigned long long bar[WS_STAGES];
+  unsigned seq;  // stage uses so far, modulo 6: use u lives in stage u % 3 with phase parity (u / 3) & 1
+};
+
 struct Cx {
   int tid, nthr;       // thread index in the compute group, group size
   int warp, nwarps, lane;
   int bar;             // named barrier id of the compute group
   float4* part;        // shared scratch, >= nwarps entries
+  WarpSmem* ws;        // this warp's staging area
+  DevState* st;        // error reporting (null in the one-kernel-per-op baseline)
+  HostCtl* hctl;
+  u64 id;              // op id, for error reports
 };
 
 struct OpEnv {
@@ -96,6 +112,62 @@ __device__ __forceinline__ void st1(u64 base, long long i, float v) {
   else
     reinterpret_cast<unsigned short*>(base)[i] = f2bf(v);
 }
+
+// ------------------------------------------------------------------ staged (shared-memory) access
+__device__ __forceinline__ void lds8_f32(unsigned a, float (&v)[8]) {
+  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]) : "r"(a));
+  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7]) : "r"(a + 16));
+}
+// 8 elements at shared byte address a
+template <int DT>
+__device__ __forceinline__ void lds8(unsigned a, float (&v)[8]) {
+  if (DT == 0) {
+    lds8_f32(a, v);
+  } else {
+    unsigned w0, w1, w2, w3;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3) : "r"(a));
+    const unsigned w[4] = {w0, w1, w2, w3};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[2 * j] = __uint_as_float(w[j] << 16);
+      v[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+    }
+  }
+}
+template <int DT>
+__device__ __forceinline__ float lds1(unsigned a) {
+  if (DT == 0) {
+    float f;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(f) : "r"(a));
+    return f;
+  }
+  unsigned short h;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(h) : "r"(a));
+  return bf2f(h);
+}
+
+// Waits for stage use u of this warp's staging area, bounded by one second;
+// a copy that never lands is reported (GPUOS_ETIMEDOUT) instead of hanging.
+static __device__ __noinline__ void ws_wait_fail(const Cx cx) {
+  if (cx.lane == 0) raise_error(cx.st, cx.hctl, GPUOS_ETIMEDOUT, cx.id);
+}
+__device__ __forceinline__ void ws_wait(const Cx& cx, unsigned u) {
+  unsigned long long* b = &cx.ws->bar[u % WS_STAGES];
+  const unsigned par = (u / WS_STAGES) & 1u;
+  if (mbar_try_wait(b, par)) return;
+  const u64 t0 = globaltimer();
+  for (unsigned spins = 0;; ++spins) {
+    if (mbar_try_wait(b, par)) return;
+    if ((spins & 1023) == 1023) {
+      if (cx.st && ld_relaxed_gpu(&cx.st->abort_.v)) return;  // another CTA failed: stop waiting
+      if (globaltimer() - t0 > 1000000000ull) {
+        ws_wait_fail(cx);
+        return;
+      }
+    }
+  }
+}
+__device__ __forceinline__ unsigned ws_addr(const Cx& cx, unsigned byte_off) { return smem_u32(cx.ws->buf) + byte_off; }
 
 // ------------------------------------------------------------------ scalar defs
 __device__ __forceinline__ float relu_f(float v) { return (v <= 0.0f) ? 0.0f : v; }  // NaN passes, -0 -> +0
@@ -307,6 +379,93 @@ static __device__ __noinline__ void ew_loop(const RingEntry& E, u32 item, u32 el
   }
 }
 
+// Elementwise item through this warp's staging area: the item is cut into
+// chunks of 2 KB per operand; warp w takes chunks w, w + nwarps, ...; lane 0
+// keeps three chunks in flight with bulk copies while the warp computes the
+// oldest from shared memory and stores straight to global memory. Operands
+// 0 and (if CH) 1 are staged; they must be direct (no broadcast) and 16-byte
+// aligned, as must the output. The op's ragged end (< 16 bytes) is read from
+// global memory.
+constexpr int EW_CHUNK_BYTES = WS_STAGE_BYTES / 2;
+
+template <int DT, int OPK, int CH>
+static __device__ __noinline__ void ew_stream(const RingEntry& E, u32 item, u32 elem_chunk, const Cx cx) {
+  constexpr int ES = DT == 0 ? 4 : 2;
+  constexpr int CE = EW_CHUNK_BYTES / ES;  // elements per chunk
+  const long long n = E.rows * E.cols;
+  const long long e0 = (long long)item * elem_chunk;
+  const long long e1 = min(n, e0 + (long long)elem_chunk);
+  const long long nchunks = (e1 - e0 + CE - 1) / CE;
+  const int w = cx.warp, NW = cx.nwarps, lane = cx.lane;
+  const int mine = nchunks > w ? (int)((nchunks - w + NW - 1) / NW) : 0;
+  if (mine == 0) return;
+  const unsigned base = cx.ws->seq;
+  __syncwarp();
+  auto issue = [&](int t) {  // lane 0 only
+    const long long e = e0 + (long long)(w + t * NW) * CE;
+    const long long ne = min((long long)CE, e1 - e);
+    const unsigned bytes = (unsigned)((ne * ES) & ~15ll);
+    const unsigned u = base + (unsigned)t;
+    unsigned long long* b = &cx.ws->bar[u % WS_STAGES];
+    unsigned char* dst = cx.ws->buf + (u % WS_STAGES) * WS_STAGE_BYTES;
+    mbar_arrive_expect_tx(b, CH ? 2 * bytes : bytes);
+    if (bytes) {
+      bulk_g2s(dst, reinterpret_cast<const unsigned char*>(E.in0) + e * ES, bytes, b);
+      if (CH) bulk_g2s(dst + EW_CHUNK_BYTES, reinterpret_cast<const unsigned char*>(E.in1) + e * ES, bytes, b);
+    }
+  };
+  if (lane == 0) {
+    for (int t = 0; t < mine && t < WS_STAGES; ++t) issue(t);
+  }
+  for (int t = 0; t < mine; ++t) {
+    const unsigned u = base + (unsigned)t;
+    const long long e = e0 + (long long)(w + t * NW) * CE;
+    const long long ne = min((long long)CE, e1 - e);
+    const long long staged = ((ne * ES) & ~15ll) / ES;  // elements that arrived by bulk copy
+    ws_wait(cx, u);
+    const unsigned a0 = ws_addr(cx, (u % WS_STAGES) * WS_STAGE_BYTES);
+#pragma unroll
+    for (int k = 0; k < CE / 8 / 32; ++k) {
+      const int blk = lane + 32 * k;
+      const long long eb = blk * 8;  // element offset within the chunk
+      if (eb >= ne) continue;
+      float x[8], y[8], z[8];
+      if (eb + 8 <= staged) {
+        lds8<DT>(a0 + (unsigned)(eb * ES), x);
+        if (CH) lds8<DT>(a0 + EW_CHUNK_BYTES + (unsigned)(eb * ES), y);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const long long ej = eb + j;
+          x[j] = ej < staged ? lds1<DT>(a0 + (unsigned)(ej * ES)) : (ej < ne ? ld1<DT>(E.in0, e + ej) : 0.f);
+          if (CH) y[j] = ej < staged ? lds1<DT>(a0 + EW_CHUNK_BYTES + (unsigned)(ej * ES)) : (ej < ne ? ld1<DT>(E.in1, e + ej) : 0.f);
+        }
+      }
+      if (!CH) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) y[j] = 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) z[j] = 0.f;
+      if (OPK == GPUOS_OP_EW_CHAIN) {
+        chain8(E, x, y, z);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) x[j] = ew_f<OPK>(E, x[j], y[j], 0.f);
+      }
+      if (eb + 8 <= ne) {
+        st8<DT>(E.out, e + eb, x);
+      } else {
+        for (int j = 0; j < 8 && eb + j < ne; ++j) st1<DT>(E.out, e + eb + j, x[j]);
+      }
+    }
+    __syncwarp();  // every lane is done with this stage before it is refilled
+    if (lane == 0 && t + WS_STAGES < mine) issue(t + WS_STAGES);
+  }
+  if (lane == 0) cx.ws->seq = (base + (unsigned)mine) % (2 * WS_STAGES);
+  __syncwarp();
+}
+
 __device__ __forceinline__ bool chain_calls(const RingEntry& E) {
   bool c = false;
   for (int i = 0; i < E.nmicro; ++i) c |= (E.micro[i] == GPUOS_M_GELU || E.micro[i] == GPUOS_M_SILU);
@@ -315,6 +474,31 @@ __device__ __forceinline__ bool chain_calls(const RingEntry& E) {
 
 template <int DT>
 __device__ void ew_item(const RingEntry& E, u32 item, u32 elem_chunk, const Cx& cx) {
+  const long long n = E.rows * E.cols;
+  const bool s0 = E.in_n0 == n && al16(E.in0);
+  const bool s1 = E.in_n1 == n && al16(E.in1);
+  if (s0 && al16(E.out)) {
+    bool u1 = false, u2 = false;
+    if (E.opcode == GPUOS_OP_EW_CHAIN) chain_uses(E, u1, u2);
+    const bool bin = E.opcode == GPUOS_OP_ADD || E.opcode == GPUOS_OP_MUL || E.opcode == GPUOS_OP_SILU_MUL;
+    if (!u2 && (!(bin || u1) || s1)) {
+      switch (E.opcode) {
+        case GPUOS_OP_ADD: ew_stream<DT, GPUOS_OP_ADD, 1>(E, item, elem_chunk, cx); return;
+        case GPUOS_OP_MUL: ew_stream<DT, GPUOS_OP_MUL, 1>(E, item, elem_chunk, cx); return;
+        case GPUOS_OP_SCALE: ew_stream<DT, GPUOS_OP_SCALE, 0>(E, item, elem_chunk, cx); return;
+        case GPUOS_OP_GELU: ew_stream<DT, GPUOS_OP_GELU, 0>(E, item, elem_chunk, cx); return;
+        case GPUOS_OP_RELU_AFFINE: ew_stream<DT, GPUOS_OP_RELU_AFFINE, 0>(E, item, elem_chunk, cx); return;
+        case GPUOS_OP_SILU_MUL: ew_stream<DT, GPUOS_OP_SILU_MUL, 1>(E, item, elem_chunk, cx); return;
+        default:
+          if (chain_calls(E)) break;  // fused programs with out-of-line calls keep the register path
+          if (u1)
+            ew_stream<DT, GPUOS_OP_EW_CHAIN, 1>(E, item, elem_chunk, cx);
+          else
+            ew_stream<DT, GPUOS_OP_EW_CHAIN, 0>(E, item, elem_chunk, cx);
+          return;
+      }
+    }
+  }
   switch (E.opcode) {
     case GPUOS_OP_ADD: ew_loop<DT, GPUOS_OP_ADD, EW_UNR, 1>(E, item, elem_chunk, cx); break;
     case GPUOS_OP_MUL: ew_loop<DT, GPUOS_OP_MUL, EW_UNR, 1>(E, item, elem_chunk, cx); break;
@@ -421,24 +605,46 @@ __device__ __forceinline__ void acc_warp(int op, Acc& A) {
 }
 
 // Writes the outputs of columns [c0, c1) of one row from its full statistic.
-template <int DT>
-__device__ void row_out(const RingEntry& E, int op, long long rb, long long c0, long long c1, Acc A, float K,
-                        bool vec, int lane) {
-  const long long cols = E.cols;
-  const float eps = E.s[0];
-  float p0 = 0.f, p1 = 0.f;  // per-row constants
+// Per-row constants of the output pass from the row's full statistic:
+// softmax (max, sum), RMSNorm (1/rms, -), LayerNorm (mean, 1/std).
+__device__ __forceinline__ void row_consts(int op, const Acc& A, float K, long long cols, float eps, float& p0,
+                                           float& p1) {
+  p0 = 0.f;
+  p1 = 0.f;
   if (op == GPUOS_OP_SOFTMAX) {
     p0 = A.a;
     p1 = A.b;
   } else if (op == GPUOS_OP_RMSNORM) {
     p0 = 1.0f / sqrtf(A.a / (float)cols + eps);
-  } else {  // LAYERNORM
+  } else if (op == GPUOS_OP_LAYERNORM) {
     const float mean_d = A.a / (float)cols;
     float var = (A.b - A.a * mean_d) / (float)cols;
     var = fmaxf(var, 0.f);
     p0 = K + mean_d;
     p1 = 1.0f / sqrtf(var + eps);
   }
+}
+
+__device__ __forceinline__ void row_apply8(int op, float p0, float p1, const float (&x)[8], const float (&w)[8],
+                                           const float (&b)[8], float (&y)[8]) {
+  if (op == GPUOS_OP_SOFTMAX) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) y[j] = __fdiv_rn(expf(x[j] - p0), p1);
+  } else if (op == GPUOS_OP_RMSNORM) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) y[j] = __fmul_rn(__fmul_rn(x[j], p0), w[j]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) y[j] = __fmaf_rn(__fmul_rn(x[j] - p0, p1), w[j], b[j]);
+  }
+}
+
+template <int DT>
+__device__ void row_out(const RingEntry& E, int op, long long rb, long long c0, long long c1, Acc A, float K,
+                        bool vec, int lane) {
+  const long long cols = E.cols;
+  float p0, p1;  // per-row constants
+  row_consts(op, A, K, cols, E.s[0], p0, p1);
   if (vec) {
     for (long long c = c0 + (long long)lane * 8; c < c1; c += 256) {
       float x[8], y[8];
@@ -476,6 +682,227 @@ __device__ void row_out(const RingEntry& E, int op, long long rb, long long c0, 
 }
 
 constexpr int ROW_UNR = 8;
+
+// ------------------------------------------------------------------ staged row ops
+// Statistic of ne elements (a multiple of 8) staged at shared address a.
+template <int DT>
+__device__ __forceinline__ void acc_s(int op, Acc& A, unsigned a, int ne, float K, int lane) {
+  constexpr int ES = DT == 0 ? 4 : 2;
+  for (int v = lane; v * 8 < ne; v += 32) {
+    float x[8];
+    lds8<DT>(a + (unsigned)(v * 8 * ES), x);
+    acc8(op, A, x, K);
+  }
+}
+
+// Output pass of ne staged elements: x at xa, weights at wa / ba (norms), to global element go.
+template <int DT>
+__device__ __forceinline__ void row_out_s(const RingEntry& E, int op, unsigned xa, unsigned wa, unsigned ba,
+                                          long long go, int ne, float p0, float p1, int lane) {
+  constexpr int ES = DT == 0 ? 4 : 2;
+  for (int v = lane; v * 8 < ne; v += 32) {
+    float x[8], w[8], b[8], y[8];
+    lds8<DT>(xa + (unsigned)(v * 8 * ES), x);
+    if (op == GPUOS_OP_RMSNORM || op == GPUOS_OP_LAYERNORM) lds8<DT>(wa + (unsigned)(v * 8 * ES), w);
+    if (op == GPUOS_OP_LAYERNORM) lds8<DT>(ba + (unsigned)(v * 8 * ES), b);
+    row_apply8(op, p0, p1, x, w, b, y);
+    st8<DT>(E.out, go + v * 8, y);
+  }
+}
+
+// Row item with every row segment staged through this warp's staging area by
+// bulk copies: one copy brings a segment (and its weights), both passes read
+// shared memory. Segments up to 4 KB (with weights) are pipelined three deep;
+// up to 12 KB they use the whole area; longer segments stream in 4 KB chunks
+// (read twice by two-pass ops, weights then from global memory). Requires
+// 16-byte aligned tensors and cols % 8 == 0.
+template <int DT>
+static __device__ __noinline__ void row_staged(const RingEntry& E, u32 item, u32 row_chunk, const Cx cx) {
+  constexpr int ES = DT == 0 ? 4 : 2;
+  const long long rows = E.rows, cols = E.cols;
+  const long long rpi = rows_per_item(cols, row_chunk);
+  const long long r0 = (long long)item * rpi;
+  const int R = (int)min(rpi, rows - r0);
+  const int op = E.opcode;
+  int S = 1;
+  while (2 * S * R <= cx.nwarps && cols / (2 * S) >= 256) S *= 2;
+  long long seg = (cols + S - 1) / S;
+  seg = (seg + 7) & ~7ll;
+  const int tasks = R * S;
+  const int nwv = op == GPUOS_OP_RMSNORM ? 1 : (op == GPUOS_OP_LAYERNORM ? 2 : 0);
+  const bool stats_only = (op == GPUOS_OP_ROWSUM || op == GPUOS_OP_ROWMAX);
+  const long long unitb = seg * ES * (1 + nwv);
+  const int mode = unitb <= WS_STAGE_BYTES ? 0 : (unitb <= WS_BYTES ? 1 : 2);
+  const int lane = cx.lane, w = cx.warp, NW = cx.nwarps;
+  const int mine = tasks > w ? (tasks - w + NW - 1) / NW : 0;
+  const unsigned base = cx.ws->seq;
+  unsigned u = base;  // next stage use
+  __syncwarp();
+  const unsigned char* in0 = reinterpret_cast<const unsigned char*>(E.in0);
+  const unsigned char* in1 = reinterpret_cast<const unsigned char*>(E.in1);
+  const unsigned char* in2 = reinterpret_cast<const unsigned char*>(E.in2);
+
+  if (mode <= 1) {
+    // one stage use per task; mode 0 keeps three tasks in flight
+    auto issue = [&](int i) {  // lane 0
+      const int t = w + i * NW;
+      const int row = t / S, sg = t % S;
+      const long long c0 = (long long)sg * seg, c1 = min(cols, c0 + seg);
+      const unsigned xb = (unsigned)((c1 - c0) * ES);
+      const unsigned uu = base + (unsigned)i;
+      unsigned long long* b = &cx.ws->bar[uu % WS_STAGES];
+      unsigned char* dst = cx.ws->buf + (mode == 0 ? (uu % WS_STAGES) * WS_STAGE_BYTES : 0);
+      mbar_arrive_expect_tx(b, xb * (unsigned)(1 + nwv));
+      bulk_g2s(dst, in0 + ((r0 + row) * cols + c0) * ES, xb, b);
+      if (nwv >= 1) bulk_g2s(dst + xb, in1 + c0 * ES, xb, b);
+      if (nwv >= 2) bulk_g2s(dst + 2 * xb, in2 + c0 * ES, xb, b);
+    };
+    const int depth = mode == 0 ? WS_STAGES : 1;
+    if (lane == 0) {
+      for (int i = 0; i < mine && i < depth; ++i) issue(i);
+    }
+    for (int i = 0; i < mine; ++i) {
+      const int t = w + i * NW;
+      const int row = t / S, sg = t % S;
+      const long long c0 = (long long)sg * seg, c1 = min(cols, c0 + seg);
+      const int ne = (int)(c1 - c0);
+      const unsigned uu = base + (unsigned)i;
+      const unsigned xa = ws_addr(cx, mode == 0 ? (uu % WS_STAGES) * WS_STAGE_BYTES : 0);
+      const unsigned wa = xa + (unsigned)(ne * ES), ba = xa + 2u * (unsigned)(ne * ES);
+      const float K = op == GPUOS_OP_LAYERNORM ? ld1<DT>(E.in0, (r0 + row) * cols) : 0.f;
+      ws_wait(cx, uu);
+      Acc A = acc_init(op);
+      acc_s<DT>(op, A, xa, ne, K, lane);
+      acc_warp(op, A);
+      if (S == 1) {
+        if (stats_only) {
+          if (lane == 0) st1<DT>(E.out, r0 + row, A.a);
+        } else {
+          float p0, p1;
+          row_consts(op, A, K, cols, E.s[0], p0, p1);
+          row_out_s<DT>(E, op, xa, wa, ba, (r0 + row) * cols + c0, ne, p0, p1, lane);
+        }
+      } else if (lane == 0) {
+        cx.part[t] = make_float4(A.a, A.b, K, 0.f);
+      }
+      __syncwarp();
+      if (lane == 0 && i + depth < mine) issue(i + depth);
+    }
+    u = base + (unsigned)mine;
+    if (S > 1) {  // at most one task per warp here; its segment is still staged
+      cx_sync(cx);
+      if (mine == 1) {
+        const int t = w;
+        const int row = t / S, sg = t % S;
+        const long long c0 = (long long)sg * seg, c1 = min(cols, c0 + seg);
+        const int ne = (int)(c1 - c0);
+        const float4 q0 = cx.part[row * S];
+        Acc A{q0.x, q0.y};
+        const float K = q0.z;
+        for (int j = 1; j < S; ++j) {
+          const float4 q = cx.part[row * S + j];
+          acc_merge(op, A, Acc{q.x, q.y});
+        }
+        if (stats_only) {
+          if (sg == 0 && lane == 0) st1<DT>(E.out, r0 + row, A.a);
+        } else {
+          const unsigned xa = ws_addr(cx, mode == 0 ? (base % WS_STAGES) * WS_STAGE_BYTES : 0);
+          float p0, p1;
+          row_consts(op, A, K, cols, E.s[0], p0, p1);
+          row_out_s<DT>(E, op, xa, xa + (unsigned)(ne * ES), xa + 2u * (unsigned)(ne * ES), (r0 + row) * cols + c0,
+                        ne, p0, p1, lane);
+        }
+      }
+    }
+  } else {
+    // long segments: stream x in 4 KB chunks through the three stages
+    constexpr long long CHE = WS_STAGE_BYTES / ES;  // elements per chunk
+    auto issue_chunk = [&](unsigned uu, long long gel, unsigned bytes) {  // lane 0
+      unsigned long long* b = &cx.ws->bar[uu % WS_STAGES];
+      mbar_arrive_expect_tx(b, bytes);
+      bulk_g2s(cx.ws->buf + (uu % WS_STAGES) * WS_STAGE_BYTES, in0 + gel * ES, bytes, b);
+    };
+    // streams segment [gs, gs + ne) once; pass 0 accumulates, pass 1 writes outputs
+    auto stream_pass = [&](long long gs, long long ne, int pass, Acc& A, float K, float p0, float p1,
+                           long long cbase) {
+      const int nch = (int)((ne + CHE - 1) / CHE);
+      const unsigned ub = u;
+      if (lane == 0) {
+        for (int k = 0; k < nch && k < WS_STAGES; ++k)
+          issue_chunk(ub + (unsigned)k, gs + k * CHE, (unsigned)(min(CHE, ne - k * CHE) * ES));
+      }
+      for (int k = 0; k < nch; ++k) {
+        const unsigned uu = ub + (unsigned)k;
+        const int ce = (int)min(CHE, ne - k * CHE);
+        ws_wait(cx, uu);
+        const unsigned xa = ws_addr(cx, (uu % WS_STAGES) * WS_STAGE_BYTES);
+        if (pass == 0) {
+          acc_s<DT>(op, A, xa, ce, K, lane);
+        } else {
+          for (int v = lane; v * 8 < ce; v += 32) {
+            float x[8], wv[8], bv[8], y[8];
+            lds8<DT>(xa + (unsigned)(v * 8 * ES), x);
+            const long long c = cbase + k * CHE + v * 8;  // column
+            if (op == GPUOS_OP_RMSNORM || op == GPUOS_OP_LAYERNORM) ld8<DT>(E.in1, c, wv);
+            if (op == GPUOS_OP_LAYERNORM) ld8<DT>(E.in2, c, bv);
+            row_apply8(op, p0, p1, x, wv, bv, y);
+            st8<DT>(E.out, gs + k * CHE + v * 8, y);
+          }
+        }
+        __syncwarp();
+        if (lane == 0 && k + WS_STAGES < nch)
+          issue_chunk(ub + (unsigned)(k + WS_STAGES), gs + (k + WS_STAGES) * CHE,
+                      (unsigned)(min(CHE, ne - (k + WS_STAGES) * CHE) * ES));
+      }
+      u = ub + (unsigned)nch;
+    };
+    for (int i = 0; i < mine; ++i) {
+      const int t = w + i * NW;
+      const int row = t / S, sg = t % S;
+      const long long c0 = (long long)sg * seg, c1 = min(cols, c0 + seg);
+      const long long gs = (r0 + row) * cols + c0;
+      const float K = op == GPUOS_OP_LAYERNORM ? ld1<DT>(E.in0, (r0 + row) * cols) : 0.f;
+      Acc A = acc_init(op);
+      stream_pass(gs, c1 - c0, 0, A, K, 0.f, 0.f, c0);
+      acc_warp(op, A);
+      if (S == 1) {
+        if (stats_only) {
+          if (lane == 0) st1<DT>(E.out, r0 + row, A.a);
+        } else {
+          float p0, p1;
+          row_consts(op, A, K, cols, E.s[0], p0, p1);
+          stream_pass(gs, c1 - c0, 1, A, K, p0, p1, c0);
+        }
+      } else if (lane == 0) {
+        cx.part[t] = make_float4(A.a, A.b, K, 0.f);
+      }
+    }
+    if (S > 1) {
+      cx_sync(cx);
+      if (mine == 1) {
+        const int t = w;
+        const int row = t / S, sg = t % S;
+        const long long c0 = (long long)sg * seg, c1 = min(cols, c0 + seg);
+        const float4 q0 = cx.part[row * S];
+        Acc A{q0.x, q0.y};
+        const float K = q0.z;
+        for (int j = 1; j < S; ++j) {
+          const float4 q = cx.part[row * S + j];
+          acc_merge(op, A, Acc{q.x, q.y});
+        }
+        if (stats_only) {
+          if (sg == 0 && lane == 0) st1<DT>(E.out, r0 + row, A.a);
+        } else {
+          float p0, p1;
+          row_consts(op, A, K, cols, E.s[0], p0, p1);
+          stream_pass((r0 + row) * cols + c0, c1 - c0, 1, A, K, p0, p1, c0);
+        }
+      }
+    }
+  }
+  if (lane == 0) cx.ws->seq = u % (2 * WS_STAGES);
+  __syncwarp();
+}
 
 // cos and sin of pos * base^(-2i/cols), in double.
 static __device__ __noinline__ double2 rotary_cs(double base, long long i, long long cols, int pos) {
@@ -608,10 +1035,20 @@ __device__ __forceinline__ void run_item(const RingEntry& E, u32 item, u32 elem_
       return;
     }
     if (op_is_row(op)) {
-      if (E.dtype == 0)
+      bool staged = op != GPUOS_OP_ROTARY && al16(E.in0) && (E.cols % 8) == 0;
+      if (op == GPUOS_OP_SOFTMAX || op == GPUOS_OP_RMSNORM || op == GPUOS_OP_LAYERNORM) staged = staged && al16(E.out);
+      if (op == GPUOS_OP_RMSNORM || op == GPUOS_OP_LAYERNORM) staged = staged && al16(E.in1);
+      if (op == GPUOS_OP_LAYERNORM) staged = staged && al16(E.in2);
+      if (staged) {
+        if (E.dtype == 0)
+          row_staged<0>(E, item, row_chunk, cx);
+        else
+          row_staged<1>(E, item, row_chunk, cx);
+      } else if (E.dtype == 0) {
         row_item<0>(E, item, row_chunk, cx);
-      else
+      } else {
         row_item<1>(E, item, row_chunk, cx);
+      }
       return;
     }
   }

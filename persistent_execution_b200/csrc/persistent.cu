@@ -703,7 +703,7 @@ __device__ void publisher(const KParams& p, Smem* S) {
 }
 
 // ------------------------------------------------------------------ compute warps
-__device__ void compute(const KParams& p, Smem* S, int warp, int lane) {
+__device__ void compute(const KParams& p, Smem* S, WarpSmem* W, int warp, int lane) {
   Cx cx;
   cx.tid = threadIdx.x - 64;
   cx.nthr = NCW * 32;
@@ -712,6 +712,10 @@ __device__ void compute(const KParams& p, Smem* S, int warp, int lane) {
   cx.lane = lane;
   cx.bar = 1;
   cx.part = S->part;
+  cx.ws = W + (warp - 2);
+  cx.st = p.st;
+  cx.hctl = p.hctl;
+  cx.id = 0;
   const bool leader = cx.tid == 0;
   for (u64 k = 0;; ++k) {
     const u32 slot = (u32)(k % FIFO);
@@ -725,6 +729,7 @@ __device__ void compute(const KParams& p, Smem* S, int warp, int lane) {
     }
     const u64 t0 = leader ? globaltimer() : 0ull;
     OpEnv env{p.st, p.hctl, p.timeout_ns, s.id};
+    cx.id = s.id;
     run_item(s.e, s.item, p.elem_chunk, p.row_chunk, cx, env);
     cx_sync(cx);
     if (leader) {
@@ -736,8 +741,15 @@ __device__ void compute(const KParams& p, Smem* S, int warp, int lane) {
   }
 }
 
+// Dynamic shared memory: the scheduling block, then one staging area per compute warp.
+constexpr size_t SMEM_HDR = (sizeof(Smem) + 127) / 128 * 128;
+constexpr size_t PERSISTENT_SMEM = SMEM_HDR + NCW * sizeof(WarpSmem);
+static_assert(PERSISTENT_SMEM <= 227 * 1024, "fits one SM");
+
 __global__ void __launch_bounds__(NTHREADS, 1) gpuos_persistent_kernel(const KParams p) {
-  __shared__ Smem S;
+  extern __shared__ __align__(128) unsigned char dsm[];
+  Smem& S = *reinterpret_cast<Smem*>(dsm);
+  WarpSmem* W = reinterpret_cast<WarpSmem*>(dsm + SMEM_HDR);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     S.ncomp = 0;
@@ -746,6 +758,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) gpuos_persistent_kernel(const KPa
       mbar_init(&S.done_bar[i], 1);
       mbar_init(&S.free_bar[i], 1);
     }
+    for (int wi = 0; wi < NCW; ++wi) {
+      W[wi].seq = 0;
+      for (int j = 0; j < WS_STAGES; ++j) mbar_init(&W[wi].bar[j], 1);
+    }
+    fence_mbar_init();
   }
   __syncthreads();
   if (warp == 0) {
@@ -754,7 +771,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gpuos_persistent_kernel(const KPa
   } else if (warp == 1) {
     if (lane == 0) publisher(p, &S);
   } else {
-    compute(p, &S, warp, lane);
+    compute(p, &S, W, warp, lane);
   }
 }
 
@@ -802,7 +819,13 @@ int launch_session(const KParams& p, u64 head, u64 big_init, void* stream) {
   gpuos_reset_kernel<<<64, 256, 0, s>>>(p, head, big_init);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return (int)e;
-  gpuos_persistent_kernel<<<p.grid, NTHREADS, 0, s>>>(p);
+  static bool attr_set = false;  // per process; the attribute is per function, not per device
+  if (!attr_set) {
+    e = cudaFuncSetAttribute(gpuos_persistent_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PERSISTENT_SMEM);
+    if (e != cudaSuccess) return (int)e;
+    attr_set = true;
+  }
+  gpuos_persistent_kernel<<<p.grid, NTHREADS, PERSISTENT_SMEM, s>>>(p);
   return (int)cudaGetLastError();
 }
 

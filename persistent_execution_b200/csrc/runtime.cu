@@ -685,7 +685,7 @@ gpuos_status gpuos_graph_create(const gpuos_desc* descs, uint64_t n, uint64_t de
       kp.func = op_kernel_fn();
       kp.gridDim = dim3(gx);
       kp.blockDim = dim3(bx);
-      kp.sharedMemBytes = 0;
+      kp.sharedMemBytes = (unsigned)op_smem_bytes();
       kp.kernelParams = args;
       cudaGraphNode_t deps[2];
       size_t nd = 0;
