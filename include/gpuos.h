@@ -136,6 +136,7 @@ typedef struct gpuos_config {
 
 #define GPUOS_CFG_NO_AUTOSTART 1u /* gpuos_create_ex does not launch the kernel */
 #define GPUOS_CFG_TRACE 2u        /* record a per-op event log (gpuos_trace_read) */
+#define GPUOS_CFG_NO_BULK 4u      /* op bodies read operands with plain loads only, no bulk-copy staging */
 
 #define GPUOS_START_DRAIN 1u      /* the kernel exits once every op published before gpuos_start completed */
 

@@ -128,6 +128,7 @@ constexpr int NCW = 16;
 
 constexpr u32 KF_DRAIN = 1u;
 constexpr u32 KF_TRACE = 2u;
+constexpr u32 KF_NO_BULK = 4u;  // op bodies use register paths only (no bulk-copy staging)
 
 struct KParams {
   DevState* st;

@@ -37,6 +37,7 @@ struct Cx {
   DevState* st;        // error reporting (null in the one-kernel-per-op baseline)
   HostCtl* hctl;
   u64 id;              // op id, for error reports
+  u32 flags;           // KF_* of the launch (KF_NO_BULK: register paths only)
 };
 
 struct OpEnv {
@@ -415,6 +416,7 @@ static __device__ __noinline__ void ew_stream(const RingEntry& E, u32 item, u32 
     }
   };
   if (lane == 0) {
+    fence_proxy_async_global();  // outputs of earlier ops were written through the generic proxy
     for (int t = 0; t < mine && t < WS_STAGES; ++t) issue(t);
   }
   for (int t = 0; t < mine; ++t) {
@@ -475,7 +477,7 @@ __device__ __forceinline__ bool chain_calls(const RingEntry& E) {
 template <int DT>
 __device__ void ew_item(const RingEntry& E, u32 item, u32 elem_chunk, const Cx& cx) {
   const long long n = E.rows * E.cols;
-  const bool s0 = E.in_n0 == n && al16(E.in0);
+  const bool s0 = E.in_n0 == n && al16(E.in0) && !(cx.flags & KF_NO_BULK);
   const bool s1 = E.in_n1 == n && al16(E.in1);
   if (s0 && al16(E.out)) {
     bool u1 = false, u2 = false;
@@ -759,6 +761,7 @@ static __device__ __noinline__ void row_staged(const RingEntry& E, u32 item, u32
     };
     const int depth = mode == 0 ? WS_STAGES : 1;
     if (lane == 0) {
+      fence_proxy_async_global();
       for (int i = 0; i < mine && i < depth; ++i) issue(i);
     }
     for (int i = 0; i < mine; ++i) {
@@ -828,6 +831,7 @@ static __device__ __noinline__ void row_staged(const RingEntry& E, u32 item, u32
       const int nch = (int)((ne + CHE - 1) / CHE);
       const unsigned ub = u;
       if (lane == 0) {
+        fence_proxy_async_global();
         for (int k = 0; k < nch && k < WS_STAGES; ++k)
           issue_chunk(ub + (unsigned)k, gs + k * CHE, (unsigned)(min(CHE, ne - k * CHE) * ES));
       }
@@ -1035,7 +1039,7 @@ __device__ __forceinline__ void run_item(const RingEntry& E, u32 item, u32 elem_
       return;
     }
     if (op_is_row(op)) {
-      bool staged = op != GPUOS_OP_ROTARY && al16(E.in0) && (E.cols % 8) == 0;
+      bool staged = op != GPUOS_OP_ROTARY && al16(E.in0) && (E.cols % 8) == 0 && !(cx.flags & KF_NO_BULK);
       if (op == GPUOS_OP_SOFTMAX || op == GPUOS_OP_RMSNORM || op == GPUOS_OP_LAYERNORM) staged = staged && al16(E.out);
       if (op == GPUOS_OP_RMSNORM || op == GPUOS_OP_LAYERNORM) staged = staged && al16(E.in1);
       if (op == GPUOS_OP_LAYERNORM) staged = staged && al16(E.in2);

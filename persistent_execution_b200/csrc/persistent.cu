@@ -716,6 +716,7 @@ __device__ void compute(const KParams& p, Smem* S, WarpSmem* W, int warp, int la
   cx.st = p.st;
   cx.hctl = p.hctl;
   cx.id = 0;
+  cx.flags = p.flags;
   const bool leader = cx.tid == 0;
   for (u64 k = 0;; ++k) {
     const u32 slot = (u32)(k % FIFO);

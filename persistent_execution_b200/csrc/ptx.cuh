@@ -98,6 +98,11 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(unsigned long long* bar, u
                "r"(bytes)
                : "memory");
 }
+// Orders this thread's view of global memory (including writes it observed
+// through acquire/barrier synchronisation) before its later bulk copies,
+// which run in the async proxy.
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
 // Makes initialised mbarriers visible to the bulk-copy (async) proxy.
 __device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
 

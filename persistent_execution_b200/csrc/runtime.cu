@@ -252,7 +252,8 @@ gpuos_status start_kernel(gpuos* rt, u32 flags) {
   p.elem_chunk = rt->cfg.elem_chunk;
   p.row_chunk = rt->cfg.row_chunk;
   p.backoff_ns = rt->cfg.backoff_ns;
-  p.flags = ((flags & GPUOS_START_DRAIN) ? KF_DRAIN : 0u) | ((rt->cfg.flags & GPUOS_CFG_TRACE) ? KF_TRACE : 0u);
+  p.flags = ((flags & GPUOS_START_DRAIN) ? KF_DRAIN : 0u) | ((rt->cfg.flags & GPUOS_CFG_TRACE) ? KF_TRACE : 0u) |
+            ((rt->cfg.flags & GPUOS_CFG_NO_BULK) ? KF_NO_BULK : 0u);
   p.grid = rt->grid;
   const int e = launch_session(p, rt->published, big_init, rt->stream);
   if (e != 0) {
