@@ -187,6 +187,23 @@ static __device__ __noinline__ float silu_mul_f(float g, float u) {
   return (float)(gd / (1.0 + exp(-gd)) * (double)u);
 }
 
+// exp for softmax: the hardware 2^t approximation (ex2.approx.f32: relative
+// error about 2^-22, subnormal results kept) at t = x log2(e). Rounding t costs
+// a relative error of |t| 2^-24 ln 2 in the result, about 1e-6 at the
+// x >= -25 that softmax rows of moderate spread reach: far inside the 1e-4 bound.
+__device__ __forceinline__ float sm_exp(float x) {
+  float r;
+  asm("ex2.approx.f32 %0, %1;" : "=f"(r) : "f"(x * 1.4426950408889634f));
+  return r;
+}
+
+// silu(g) * u for bf16 outputs, whose bound (2 bf16 ulp) leaves room for fp32
+// with the hardware exp; large |g| keeps the double path.
+__device__ __forceinline__ float silu_mul_bf(float g, float u) {
+  if (fabsf(g) > 80.0f) return silu_mul_f(g, u);
+  return __fdividef(g, 1.0f + __expf(-g)) * u;
+}
+
 // Fused micro-op program over one element; the program and scalars are read
 // from the shared-memory entry (uniform across the group).
 __device__ __forceinline__ float chain_f(const RingEntry& E, float acc, float x1, float x2) {
@@ -210,14 +227,14 @@ __device__ __forceinline__ float chain_f(const RingEntry& E, float acc, float x1
   return acc;
 }
 
-template <int OPK>
+template <int OPK, int DT = 0>
 __device__ __forceinline__ float ew_f(const RingEntry& E, float x0, float x1, float x2) {
   if (OPK == GPUOS_OP_ADD) return __fadd_rn(x0, x1);
   if (OPK == GPUOS_OP_MUL) return __fmul_rn(x0, x1);
   if (OPK == GPUOS_OP_SCALE) return __fmul_rn(E.s[0], x0);
   if (OPK == GPUOS_OP_GELU) return gelu_f(x0);
   if (OPK == GPUOS_OP_RELU_AFFINE) return relu_f(__fmaf_rn(E.s[0], x0, E.s[1]));
-  if (OPK == GPUOS_OP_SILU_MUL) return silu_mul_f(x0, x1);
+  if (OPK == GPUOS_OP_SILU_MUL) return DT == 1 ? silu_mul_bf(x0, x1) : silu_mul_f(x0, x1);
   return chain_f(E, x0, x1, x2);  // GPUOS_OP_EW_CHAIN, OPK_CHAIN_CALLS
 }
 
@@ -361,7 +378,7 @@ static __device__ __noinline__ void ew_loop(const RingEntry& E, u32 item, u32 el
           chain8(E, a[u], b[u], c[u]);
         } else {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) a[u][j] = ew_f<OPK>(E, a[u][j], b[u][j], c[u][j]);
+          for (int j = 0; j < 8; ++j) a[u][j] = ew_f<OPK, DT>(E, a[u][j], b[u][j], c[u][j]);
         }
         if (all_vec || vout) {
           st8<DT>(E.out, vi << 3, a[u]);
@@ -376,7 +393,7 @@ static __device__ __noinline__ void ew_loop(const RingEntry& E, u32 item, u32 el
     const float x0 = ld1<DT>(E.in0, n0 == n ? e : (long long)umod((u64)e, (u64)n0));
     const float x1 = u1 ? ld1<DT>(E.in1, n1 == n ? e : (long long)umod((u64)e, (u64)n1)) : 0.f;
     const float x2 = u2 ? ld1<DT>(E.in2, e) : 0.f;
-    st1<DT>(E.out, e, ew_f<OPK>(E, x0, x1, x2));
+    st1<DT>(E.out, e, ew_f<OPK, DT>(E, x0, x1, x2));
   }
 }
 
@@ -453,7 +470,7 @@ static __device__ __noinline__ void ew_stream(const RingEntry& E, u32 item, u32 
         chain8(E, x, y, z);
       } else {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) x[j] = ew_f<OPK>(E, x[j], y[j], 0.f);
+        for (int j = 0; j < 8; ++j) x[j] = ew_f<OPK, DT>(E, x[j], y[j], 0.f);
       }
       if (eb + 8 <= ne) {
         st8<DT>(E.out, e + eb, x);
@@ -550,9 +567,9 @@ __device__ __forceinline__ void acc8(int op, Acc& A, const float (&x)[8], float 
     float m = A.a;
 #pragma unroll
     for (int j = 0; j < 8; ++j) m = fmaxf(m, x[j]);
-    float s = (A.a == -INFINITY) ? 0.f : A.b * expf(A.a - m);
+    float s = (A.a == -INFINITY) ? 0.f : A.b * sm_exp(A.a - m);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) s += expf(x[j] - m);
+    for (int j = 0; j < 8; ++j) s += sm_exp(x[j] - m);
     A.a = m;
     A.b = s;
   } else if (op == GPUOS_OP_RMSNORM) {
@@ -574,7 +591,7 @@ __device__ __forceinline__ void acc1(int op, Acc& A, float x, float K) {
     A.a = fmaxf(A.a, x);
   } else if (op == GPUOS_OP_SOFTMAX) {
     const float m = fmaxf(A.a, x);
-    A.b = ((A.a == -INFINITY) ? 0.f : A.b * expf(A.a - m)) + expf(x - m);
+    A.b = ((A.a == -INFINITY) ? 0.f : A.b * sm_exp(A.a - m)) + sm_exp(x - m);
     A.a = m;
   } else if (op == GPUOS_OP_RMSNORM) {
     A.a = __fmaf_rn(x, x, A.a);
@@ -590,7 +607,7 @@ __device__ __forceinline__ void acc_merge(int op, Acc& A, const Acc& B) {
   } else if (op == GPUOS_OP_SOFTMAX) {
     const float m = fmaxf(A.a, B.a);
     if (m != -INFINITY) {
-      A.b = A.b * expf(A.a - m) + B.b * expf(B.a - m);
+      A.b = A.b * sm_exp(A.a - m) + B.b * sm_exp(B.a - m);
       A.a = m;
     }
   } else {
@@ -615,7 +632,7 @@ __device__ __forceinline__ void row_consts(int op, const Acc& A, float K, long l
   p1 = 0.f;
   if (op == GPUOS_OP_SOFTMAX) {
     p0 = A.a;
-    p1 = A.b;
+    p1 = 1.0f / A.b;  // one division per row; outputs multiply
   } else if (op == GPUOS_OP_RMSNORM) {
     p0 = 1.0f / sqrtf(A.a / (float)cols + eps);
   } else if (op == GPUOS_OP_LAYERNORM) {
@@ -631,7 +648,7 @@ __device__ __forceinline__ void row_apply8(int op, float p0, float p1, const flo
                                            const float (&b)[8], float (&y)[8]) {
   if (op == GPUOS_OP_SOFTMAX) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) y[j] = __fdiv_rn(expf(x[j] - p0), p1);
+    for (int j = 0; j < 8; ++j) y[j] = __fmul_rn(sm_exp(x[j] - p0), p1);
   } else if (op == GPUOS_OP_RMSNORM) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) y[j] = __fmul_rn(__fmul_rn(x[j], p0), w[j]);
@@ -641,9 +658,33 @@ __device__ __forceinline__ void row_apply8(int op, float p0, float p1, const flo
   }
 }
 
+// Columns [c0, c1) of a row starting at element rb of base split as
+// [c0, ca) | [ca, cb) | [cb, c1), the middle 16-byte aligned and a multiple of
+// 8 elements long (head and tail shorter than 8).
+struct RowSplit {
+  long long ca, cb;
+};
 template <int DT>
-__device__ void row_out(const RingEntry& E, int op, long long rb, long long c0, long long c1, Acc A, float K,
+__device__ __forceinline__ RowSplit row_split(u64 base, long long rb, long long c0, long long c1) {
+  constexpr int esz = DT == 0 ? 4 : 2;
+  const u64 a = base + (u64)(rb + c0) * esz;
+  long long head = (long long)(((16u - (unsigned)(a & 15)) & 15u) / esz);
+  if (head > c1 - c0) head = c1 - c0;
+  const long long ca = c0 + head;
+  return RowSplit{ca, ca + ((c1 - ca) / 8) * 8};
+}
+
+template <int DT>
+__device__ __forceinline__ float row_apply1(const RingEntry& E, int op, float p0, float p1, float x, long long c) {
+  if (op == GPUOS_OP_SOFTMAX) return __fmul_rn(sm_exp(x - p0), p1);
+  if (op == GPUOS_OP_RMSNORM) return __fmul_rn(__fmul_rn(x, p0), ld1<DT>(E.in1, c));
+  return __fmaf_rn(__fmul_rn(x - p0, p1), ld1<DT>(E.in1, c), ld1<DT>(E.in2, c));
+}
+
+template <int DT, int OP>
+static __device__ __noinline__ void row_out(const RingEntry& E, int, long long rb, long long c0, long long c1, Acc A, float K,
                         bool vec, int lane) {
+  constexpr int op = OP;
   const long long cols = E.cols;
   float p0, p1;  // per-row constants
   row_consts(op, A, K, cols, E.s[0], p0, p1);
@@ -653,7 +694,7 @@ __device__ void row_out(const RingEntry& E, int op, long long rb, long long c0, 
       ld8<DT>(E.in0, rb + c, x);
       if (op == GPUOS_OP_SOFTMAX) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) y[j] = __fdiv_rn(expf(x[j] - p0), p1);
+        for (int j = 0; j < 8; ++j) y[j] = __fmul_rn(sm_exp(x[j] - p0), p1);
       } else if (op == GPUOS_OP_RMSNORM) {
         float w[8];
         ld8<DT>(E.in1, c, w);
@@ -669,16 +710,42 @@ __device__ void row_out(const RingEntry& E, int op, long long rb, long long c0, 
       st8<DT>(E.out, rb + c, y);
     }
   } else {
-    for (long long c = c0 + lane; c < c1; c += 32) {
-      const float x = ld1<DT>(E.in0, rb + c);
-      float y;
-      if (op == GPUOS_OP_SOFTMAX)
-        y = __fdiv_rn(expf(x - p0), p1);
-      else if (op == GPUOS_OP_RMSNORM)
-        y = __fmul_rn(__fmul_rn(x, p0), ld1<DT>(E.in1, c));
-      else
-        y = __fmaf_rn(__fmul_rn(x - p0, p1), ld1<DT>(E.in1, c), ld1<DT>(E.in2, c));
-      st1<DT>(E.out, rb + c, y);
+    // Unaligned row start. When the output (and the weights) sit at the same
+    // offset modulo 16 bytes as the input row, the middle goes as ld8/st8.
+    constexpr long long esz = DT == 0 ? 4 : 2;
+    const RowSplit sp = row_split<DT>(E.in0, rb, c0, c1);
+    const u64 shift = E.in0 + (u64)(rb * esz);
+    bool pv = ((E.out - E.in0) & 15ull) == 0;
+    if (op != GPUOS_OP_SOFTMAX) pv = pv && ((E.in1 - shift) & 15ull) == 0;
+    if (op == GPUOS_OP_LAYERNORM) pv = pv && ((E.in2 - shift) & 15ull) == 0;
+    if (pv) {
+      if (lane < sp.ca - c0) {
+        const long long c = c0 + lane;
+        st1<DT>(E.out, rb + c, row_apply1<DT>(E, op, p0, p1, ld1<DT>(E.in0, rb + c), c));
+      }
+      if (lane < c1 - sp.cb) {
+        const long long c = sp.cb + lane;
+        st1<DT>(E.out, rb + c, row_apply1<DT>(E, op, p0, p1, ld1<DT>(E.in0, rb + c), c));
+      }
+      for (long long c = sp.ca + (long long)lane * 8; c < sp.cb; c += 256) {
+        float x[8], w[8], b[8], y[8];
+        ld8<DT>(E.in0, rb + c, x);
+        if (op != GPUOS_OP_SOFTMAX) ld8<DT>(E.in1, c, w);
+        if (op == GPUOS_OP_LAYERNORM) ld8<DT>(E.in2, c, b);
+        row_apply8(op, p0, p1, x, w, b, y);
+        st8<DT>(E.out, rb + c, y);
+      }
+    } else {
+      // Element at a time, eight loads issued before the first store.
+      long long c = c0 + lane;
+      for (; c + 7 * 32 < c1; c += 256) {
+        float x[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) x[j] = ld1<DT>(E.in0, rb + c + 32 * j);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) st1<DT>(E.out, rb + c + 32 * j, row_apply1<DT>(E, op, p0, p1, x[j], c + 32 * j));
+      }
+      for (; c < c1; c += 32) st1<DT>(E.out, rb + c, row_apply1<DT>(E, op, p0, p1, ld1<DT>(E.in0, rb + c), c));
     }
   }
 }
@@ -718,14 +785,14 @@ __device__ __forceinline__ void row_out_s(const RingEntry& E, int op, unsigned x
 // up to 12 KB they use the whole area; longer segments stream in 4 KB chunks
 // (read twice by two-pass ops, weights then from global memory). Requires
 // 16-byte aligned tensors and cols % 8 == 0.
-template <int DT>
+template <int DT, int OP>
 static __device__ __noinline__ void row_staged(const RingEntry& E, u32 item, u32 row_chunk, const Cx cx) {
   constexpr int ES = DT == 0 ? 4 : 2;
   const long long rows = E.rows, cols = E.cols;
   const long long rpi = rows_per_item(cols, row_chunk);
   const long long r0 = (long long)item * rpi;
   const int R = (int)min(rpi, rows - r0);
-  const int op = E.opcode;
+  constexpr int op = OP;
   int S = 1;
   while (2 * S * R <= cx.nwarps && cols / (2 * S) >= 256) S *= 2;
   long long seg = (cols + S - 1) / S;
@@ -922,10 +989,16 @@ static __device__ __noinline__ void rotary_item(const RingEntry& E, long long r0
   const long long cols = E.cols, half = cols / 2;
   const long long total = (long long)R * half;
   const double base = (double)E.s[0];
+  long long ti = -1;  // the column pair whose angle is in cs, sn
+  double cs = 0.0, sn = 0.0;
   for (long long p = cx.tid; p < total; p += cx.nthr) {
     const long long row = p / half, i = p % half;
-    const double2 t = rotary_cs(base, i, cols, E.pos);
-    const double cs = t.x, sn = t.y;
+    if (i != ti) {  // the angle depends on the column pair only
+      const double2 t = rotary_cs(base, i, cols, E.pos);
+      cs = t.x;
+      sn = t.y;
+      ti = i;
+    }
     const long long rb = (r0 + row) * cols;
     const double x1 = (double)ld1<DT>(E.in0, rb + i), x2 = (double)ld1<DT>(E.in0, rb + i + half);
     st1<DT>(E.out, rb + i, (float)(x1 * cs - x2 * sn));
@@ -933,14 +1006,14 @@ static __device__ __noinline__ void rotary_item(const RingEntry& E, long long r0
   }
 }
 
-template <int DT>
+template <int DT, int OP>
 static __device__ __noinline__ void row_item(const RingEntry& E, u32 item, u32 row_chunk, const Cx cx) {
   const long long rows = E.rows, cols = E.cols;
   const long long rpi = rows_per_item(cols, row_chunk);
   const long long r0 = (long long)item * rpi;
   const int R = (int)min(rpi, rows - r0);
-  const int op = E.opcode;
-  if (op == GPUOS_OP_ROTARY) {
+  constexpr int op = OP;
+  if constexpr (op == GPUOS_OP_ROTARY) {
     rotary_item<DT>(E, r0, R, cx);
     return;
   }
@@ -976,14 +1049,32 @@ static __device__ __noinline__ void row_item(const RingEntry& E, u32 item, u32 r
         acc8(op, A, x, K);
       }
     } else {
-      for (long long c = c0 + cx.lane; c < c1; c += 32) acc1(op, A, ld1<DT>(E.in0, rb + c), K);
+      // Row start not 16-byte aligned (ragged lengths): the lanes take the
+      // few head and tail elements one each, the aligned middle as ld8.
+      const RowSplit sp = row_split<DT>(E.in0, rb, c0, c1);
+      if (cx.lane < sp.ca - c0) acc1(op, A, ld1<DT>(E.in0, rb + c0 + cx.lane), K);
+      if (cx.lane < c1 - sp.cb) acc1(op, A, ld1<DT>(E.in0, rb + sp.cb + cx.lane), K);
+      long long c = sp.ca + (long long)cx.lane * 8;
+      constexpr int U = ROW_UNR / 2;
+      for (; c + (long long)(U - 1) * 256 < sp.cb; c += (long long)U * 256) {
+        float x[U][8];
+#pragma unroll
+        for (int u = 0; u < U; ++u) ld8<DT>(E.in0, rb + c + u * 256, x[u]);
+#pragma unroll
+        for (int u = 0; u < U; ++u) acc8(op, A, x[u], K);
+      }
+      for (; c < sp.cb; c += 256) {
+        float x[8];
+        ld8<DT>(E.in0, rb + c, x);
+        acc8(op, A, x, K);
+      }
     }
     acc_warp(op, A);
     if (S == 1) {
       if (stats_only) {
         if (cx.lane == 0) st1<DT>(E.out, r0 + row, A.a);
       } else {
-        row_out<DT>(E, op, rb, 0, cols, A, K, vec, cx.lane);
+        row_out<DT, OP>(E, op, rb, 0, cols, A, K, vec, cx.lane);
       }
     } else if (cx.lane == 0) {
       cx.part[t] = make_float4(A.a, A.b, K, 0.f);
@@ -1005,7 +1096,7 @@ static __device__ __noinline__ void row_item(const RingEntry& E, u32 item, u32 r
       if (stats_only) {
         if (sg == 0 && cx.lane == 0) st1<DT>(E.out, r0 + row, A.a);
       } else {
-        row_out<DT>(E, op, rb, c0, c1, A, K, vec, cx.lane);
+        row_out<DT, OP>(E, op, rb, c0, c1, A, K, vec, cx.lane);
       }
     }
   }
@@ -1026,6 +1117,26 @@ __device__ __forceinline__ void stall_item(const OpEnv& env, const Cx& cx) {
   }
 }
 
+// Row bodies are instantiated per opcode so that each holds one op's code.
+template <int DT, int OP>
+__device__ __forceinline__ void row_one(const RingEntry& E, u32 item, u32 row_chunk, const Cx& cx, bool staged) {
+  if (staged)
+    row_staged<DT, OP>(E, item, row_chunk, cx);
+  else
+    row_item<DT, OP>(E, item, row_chunk, cx);
+}
+template <int DT>
+__device__ __forceinline__ void row_dispatch(const RingEntry& E, u32 item, u32 row_chunk, const Cx& cx, bool staged) {
+  switch (E.opcode) {
+    case GPUOS_OP_ROWSUM: row_one<DT, GPUOS_OP_ROWSUM>(E, item, row_chunk, cx, staged); break;
+    case GPUOS_OP_ROWMAX: row_one<DT, GPUOS_OP_ROWMAX>(E, item, row_chunk, cx, staged); break;
+    case GPUOS_OP_SOFTMAX: row_one<DT, GPUOS_OP_SOFTMAX>(E, item, row_chunk, cx, staged); break;
+    case GPUOS_OP_RMSNORM: row_one<DT, GPUOS_OP_RMSNORM>(E, item, row_chunk, cx, staged); break;
+    case GPUOS_OP_LAYERNORM: row_one<DT, GPUOS_OP_LAYERNORM>(E, item, row_chunk, cx, staged); break;
+    default: row_item<DT, GPUOS_OP_ROTARY>(E, item, row_chunk, cx); break;
+  }
+}
+
 __device__ __forceinline__ void run_item(const RingEntry& E, u32 item, u32 elem_chunk, u32 row_chunk, const Cx& cx,
                                          const OpEnv& env) {
   const int op = E.opcode;
@@ -1043,16 +1154,10 @@ __device__ __forceinline__ void run_item(const RingEntry& E, u32 item, u32 elem_
       if (op == GPUOS_OP_SOFTMAX || op == GPUOS_OP_RMSNORM || op == GPUOS_OP_LAYERNORM) staged = staged && al16(E.out);
       if (op == GPUOS_OP_RMSNORM || op == GPUOS_OP_LAYERNORM) staged = staged && al16(E.in1);
       if (op == GPUOS_OP_LAYERNORM) staged = staged && al16(E.in2);
-      if (staged) {
-        if (E.dtype == 0)
-          row_staged<0>(E, item, row_chunk, cx);
-        else
-          row_staged<1>(E, item, row_chunk, cx);
-      } else if (E.dtype == 0) {
-        row_item<0>(E, item, row_chunk, cx);
-      } else {
-        row_item<1>(E, item, row_chunk, cx);
-      }
+      if (E.dtype == 0)
+        row_dispatch<0>(E, item, row_chunk, cx, staged);
+      else
+        row_dispatch<1>(E, item, row_chunk, cx, staged);
       return;
     }
   }

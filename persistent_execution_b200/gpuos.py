@@ -14,7 +14,7 @@ import os
 import numpy as np
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libgpuos.so")
+LIB_PATH = os.environ.get("GPUOS_LIB", os.path.join(HERE, "libgpuos.so"))  # override: an alternative build
 
 OK, EINVAL, EAGAIN, ETIMEDOUT, EBADOP, EDEVICE, ESTOPPED, ENOMEM = range(8)
 STATUS = ("OK", "EINVAL", "EAGAIN", "ETIMEDOUT", "EBADOP", "EDEVICE", "ESTOPPED", "ENOMEM")
