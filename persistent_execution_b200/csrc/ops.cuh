@@ -289,36 +289,77 @@ __device__ __forceinline__ void chain_uses(const RingEntry& E, bool& u1, bool& u
   }
 }
 
-constexpr int EW_UNR = 2;  // 8-element blocks in flight per thread (binary ops; unary ops use twice as many)
+constexpr int EW_UNR = 2;  // tiles in flight per warp (binary ops; unary ops use twice as many)
 
 // Pseudo-opcode: a fused program that calls an out-of-line transcendental
 // (gelu, silu) runs element by element, without the unrolled vector batch.
 constexpr int OPK_CHAIN_CALLS = 1000;
 
-// Each body is out of line: inlined together into one dispatcher, the union
-// of their unrolled register arrays would spill.
 // e mod m, in 32 bits when both fit
 __device__ __forceinline__ u64 umod(u64 a, u64 m) {
   if (((a | m) >> 32) == 0) return (u64)((u32)a % (u32)m);
   return a % m;
 }
 
-// 8 elements e..e+7 of an operand of m elements read at index (e + t) mod m:
-// one modulo per block, eight independent loads in flight.
+// Register-path tiles: a warp takes 256 consecutive elements at a time.
+// Vector layout (all operands direct and 16-byte aligned): lane l holds
+// fp32 elements 4l..4l+3 and 128+4l..128+4l+3 (two float4, each warp load
+// one contiguous 512 bytes), or bf16 elements 8l..8l+7 (one 16-byte load).
+// Scalar layout (a broadcast or unaligned operand): lane l holds elements
+// l, l+32, ..., l+224, each warp load one contiguous 128 (64) bytes.
+constexpr int EW_TILE = 256;
+
 template <int DT>
-__device__ __forceinline__ void gather8(u64 base, long long e, long long m, long long n, float (&v)[8]) {
-  long long j = (m == n) ? e : (long long)umod((u64)e, (u64)m);
+__device__ __forceinline__ void tile_ld(u64 base, long long t0, int lane, float (&v)[8]) {
+  if (DT == 0) {
+    const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + t0);
+    const float4 a = __ldcg(p + lane), b = __ldcg(p + 32 + lane);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+    ld8<1>(base, t0 + 8 * lane, v);
+  }
+}
+template <int DT>
+__device__ __forceinline__ void tile_st(u64 base, long long t0, int lane, const float (&v)[8]) {
+  if (DT == 0) {
+    float4* p = reinterpret_cast<float4*>(reinterpret_cast<float*>(base) + t0);
+    p[lane] = make_float4(v[0], v[1], v[2], v[3]);
+    p[32 + lane] = make_float4(v[4], v[5], v[6], v[7]);
+  } else {
+    st8<1>(base, t0 + 8 * lane, v);
+  }
+}
+
+// Scalar layout of one operand of m elements read at index e mod m (m == n:
+// direct). j starts at (t0 + lane) mod m and steps by step = 32 mod m.
+template <int DT>
+__device__ __forceinline__ void tile_gather(u64 base, long long t0, int lane, long long m, long long n,
+                                            long long step, long long e1, float (&v)[8]) {
+  long long j = (m == n) ? t0 + lane : (long long)umod((u64)(t0 + lane), (u64)m);
 #pragma unroll
-  for (int t = 0; t < 8; ++t) {
-    v[t] = ld1<DT>(base, j);
-    j = (j + 1 == m) ? 0 : j + 1;
+  for (int k = 0; k < 8; ++k) {
+    v[k] = (t0 + lane + 32 * k < e1) ? ld1<DT>(base, j) : 0.f;
+    j += step;
+    if (j >= m) j -= m;
+  }
+}
+
+template <int DT, int OPK>
+__device__ __forceinline__ void ew_apply8(const RingEntry& E, float (&a)[8], const float (&b)[8],
+                                          const float (&c)[8]) {
+  if (OPK == GPUOS_OP_EW_CHAIN) {
+    chain8(E, a, b, c);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) a[j] = ew_f<OPK, DT>(E, a[j], b[j], c[j]);
   }
 }
 
 // Each body is out of line: inlined together into one dispatcher, the union
 // of their unrolled register arrays would spill.
 // CH: which extra operands the body reads (bit 0: in1, bit 1: in2), or -1 to
-// decide at run time from the fused program.
+// decide at run time from the fused program. UNR: tiles in flight per warp.
 template <int DT, int OPK, int UNR, int CH>
 static __device__ __noinline__ void ew_loop(const RingEntry& E, u32 item, u32 elem_chunk, const Cx cx) {
   const long long n = E.rows * E.cols;
@@ -332,68 +373,58 @@ static __device__ __noinline__ void ew_loop(const RingEntry& E, u32 item, u32 el
     u2 = (CH & 2) != 0;
   }
   const long long n0 = E.in_n0, n1 = E.in_n1;
-  // per operand: direct 16-byte vectors, or 8-element gathers (broadcast or unaligned)
-  const bool v0d = n0 == n && al16(E.in0);
-  const bool v1d = !u1 || (n1 == n && al16(E.in1));
-  const bool v2d = !u2 || al16(E.in2);
-  const bool vout = al16(E.out);
-  const bool all_vec = v0d && v1d && v2d && vout;
-  const long long b0 = e0 >> 3, b1 = e1 >> 3;  // whole 8-element blocks of this item
-  for (long long v = b0 + cx.tid; v < b1; v += (long long)UNR * cx.nthr) {
-    float a[UNR][8], b[UNR][8], c[UNR][8];
+  const bool vec = n0 == n && al16(E.in0) && (!u1 || (n1 == n && al16(E.in1))) && (!u2 || al16(E.in2)) &&
+                   al16(E.out);
+  const int lane = cx.lane, w = cx.warp, NW = cx.nwarps;
+  const long long full = (e1 - e0) / EW_TILE, tiles = (e1 - e0 + EW_TILE - 1) / EW_TILE;
+  long long t = w;
+  if (vec) {
+    for (; t + (long long)(UNR - 1) * NW < full; t += (long long)UNR * NW) {
+      float a[UNR][8], b[UNR][8], c[UNR][8];
 #pragma unroll
-    for (int u = 0; u < UNR; ++u) {
-      const long long vi = v + (long long)u * cx.nthr;
-      if (vi < b1) {
-        const long long e = vi << 3;
-        if (all_vec || v0d)
-          ld8<DT>(E.in0, e, a[u]);
-        else
-          gather8<DT>(E.in0, e, n0, n, a[u]);
-        if (u1) {
-          if (all_vec || (n1 == n && al16(E.in1)))
-            ld8<DT>(E.in1, e, b[u]);
-          else
-            gather8<DT>(E.in1, e, n1, n, b[u]);
-        } else {
+      for (int u = 0; u < UNR; ++u) {
+        const long long t0 = e0 + (t + (long long)u * NW) * EW_TILE;
+        tile_ld<DT>(E.in0, t0, lane, a[u]);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) b[u][j] = 0.f;
-        }
-        if (u2) {
-          if (all_vec || v2d)
-            ld8<DT>(E.in2, e, c[u]);
-          else
-            gather8<DT>(E.in2, e, n, n, c[u]);
-        } else {
+        for (int j = 0; j < 8; ++j) b[u][j] = c[u][j] = 0.f;
+        if (u1) tile_ld<DT>(E.in1, t0, lane, b[u]);
+        if (u2) tile_ld<DT>(E.in2, t0, lane, c[u]);
+      }
 #pragma unroll
-          for (int j = 0; j < 8; ++j) c[u][j] = 0.f;
-        }
+      for (int u = 0; u < UNR; ++u) {
+        ew_apply8<DT, OPK>(E, a[u], b[u], c[u]);
+        tile_st<DT>(E.out, e0 + (t + (long long)u * NW) * EW_TILE, lane, a[u]);
       }
     }
+    for (; t < full; t += NW) {
+      const long long t0 = e0 + t * EW_TILE;
+      float a[8], b[8], c[8];
+      tile_ld<DT>(E.in0, t0, lane, a);
 #pragma unroll
-    for (int u = 0; u < UNR; ++u) {
-      const long long vi = v + (long long)u * cx.nthr;
-      if (vi < b1) {
-        if (OPK == GPUOS_OP_EW_CHAIN) {
-          chain8(E, a[u], b[u], c[u]);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) a[u][j] = ew_f<OPK, DT>(E, a[u][j], b[u][j], c[u][j]);
-        }
-        if (all_vec || vout) {
-          st8<DT>(E.out, vi << 3, a[u]);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) st1<DT>(E.out, (vi << 3) + j, a[u][j]);
-        }
-      }
+      for (int j = 0; j < 8; ++j) b[j] = c[j] = 0.f;
+      if (u1) tile_ld<DT>(E.in1, t0, lane, b);
+      if (u2) tile_ld<DT>(E.in2, t0, lane, c);
+      ew_apply8<DT, OPK>(E, a, b, c);
+      tile_st<DT>(E.out, t0, lane, a);
     }
+    // t is now the first tile >= full that this warp owns: the partial last
+    // tile, if any, takes the scalar layout below
   }
-  for (long long e = (b1 << 3) + cx.tid; e < e1; e += cx.nthr) {  // ragged tail (< 8 elements)
-    const float x0 = ld1<DT>(E.in0, n0 == n ? e : (long long)umod((u64)e, (u64)n0));
-    const float x1 = u1 ? ld1<DT>(E.in1, n1 == n ? e : (long long)umod((u64)e, (u64)n1)) : 0.f;
-    const float x2 = u2 ? ld1<DT>(E.in2, e) : 0.f;
-    st1<DT>(E.out, e, ew_f<OPK, DT>(E, x0, x1, x2));
+  const long long s0 = n0 < n ? 32 % n0 : 32, s1 = (u1 && n1 < n) ? 32 % n1 : 32;
+  for (; t < tiles; t += NW) {
+    const long long t0 = e0 + t * EW_TILE;
+    float a[8], b[8], c[8];
+    tile_gather<DT>(E.in0, t0, lane, n0, n, s0, e1, a);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) b[j] = c[j] = 0.f;
+    if (u1) tile_gather<DT>(E.in1, t0, lane, n1, n, s1, e1, b);
+    if (u2) tile_gather<DT>(E.in2, t0, lane, n, n, 32, e1, c);
+    ew_apply8<DT, OPK>(E, a, b, c);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const long long e = t0 + lane + 32 * k;
+      if (e < e1) st1<DT>(E.out, e, a[k]);
+    }
   }
 }
 
@@ -658,6 +689,32 @@ __device__ __forceinline__ void row_apply8(int op, float p0, float p1, const flo
   }
 }
 
+// Folds columns [lo, hi) of a row (element rb + lo 16-byte aligned, hi - lo
+// a multiple of 8) into A: whole 256-column tiles in the tile layout, U at a
+// time, the rest as 8 consecutive columns per lane.
+template <int DT, int U>
+__device__ __forceinline__ void acc_span(int op, Acc& A, float K, u64 base, long long rb, long long lo, long long hi,
+                                         int lane) {
+  long long c = lo;
+  for (; c + (long long)U * EW_TILE <= hi; c += (long long)U * EW_TILE) {
+    float x[U][8];
+#pragma unroll
+    for (int u = 0; u < U; ++u) tile_ld<DT>(base, rb + c + u * EW_TILE, lane, x[u]);
+#pragma unroll
+    for (int u = 0; u < U; ++u) acc8(op, A, x[u], K);
+  }
+  for (; c + EW_TILE <= hi; c += EW_TILE) {
+    float x[8];
+    tile_ld<DT>(base, rb + c, lane, x);
+    acc8(op, A, x, K);
+  }
+  for (c += (long long)lane * 8; c < hi; c += EW_TILE) {
+    float x[8];
+    ld8<DT>(base, rb + c, x);
+    acc8(op, A, x, K);
+  }
+}
+
 // Columns [c0, c1) of a row starting at element rb of base split as
 // [c0, ca) | [ca, cb) | [cb, c1), the middle 16-byte aligned and a multiple of
 // 8 elements long (head and tail shorter than 8).
@@ -681,6 +738,30 @@ __device__ __forceinline__ float row_apply1(const RingEntry& E, int op, float p0
   return __fmaf_rn(__fmul_rn(x - p0, p1), ld1<DT>(E.in1, c), ld1<DT>(E.in2, c));
 }
 
+// Writes the outputs of columns [lo, hi) (same alignment rule as acc_span):
+// input row, weights and output read and written in one layout.
+template <int DT, int OP>
+__device__ __forceinline__ void out_span(const RingEntry& E, float p0, float p1, long long rb, long long lo,
+                                         long long hi, int lane) {
+  long long c = lo;
+  for (; c + EW_TILE <= hi; c += EW_TILE) {
+    float x[8], w[8], b[8], y[8];
+    tile_ld<DT>(E.in0, rb + c, lane, x);
+    if (OP != GPUOS_OP_SOFTMAX) tile_ld<DT>(E.in1, c, lane, w);
+    if (OP == GPUOS_OP_LAYERNORM) tile_ld<DT>(E.in2, c, lane, b);
+    row_apply8(OP, p0, p1, x, w, b, y);
+    tile_st<DT>(E.out, rb + c, lane, y);
+  }
+  for (c += (long long)lane * 8; c < hi; c += EW_TILE) {
+    float x[8], w[8], b[8], y[8];
+    ld8<DT>(E.in0, rb + c, x);
+    if (OP != GPUOS_OP_SOFTMAX) ld8<DT>(E.in1, c, w);
+    if (OP == GPUOS_OP_LAYERNORM) ld8<DT>(E.in2, c, b);
+    row_apply8(OP, p0, p1, x, w, b, y);
+    st8<DT>(E.out, rb + c, y);
+  }
+}
+
 template <int DT, int OP>
 static __device__ __noinline__ void row_out(const RingEntry& E, int, long long rb, long long c0, long long c1, Acc A, float K,
                         bool vec, int lane) {
@@ -689,26 +770,7 @@ static __device__ __noinline__ void row_out(const RingEntry& E, int, long long r
   float p0, p1;  // per-row constants
   row_consts(op, A, K, cols, E.s[0], p0, p1);
   if (vec) {
-    for (long long c = c0 + (long long)lane * 8; c < c1; c += 256) {
-      float x[8], y[8];
-      ld8<DT>(E.in0, rb + c, x);
-      if (op == GPUOS_OP_SOFTMAX) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) y[j] = __fmul_rn(sm_exp(x[j] - p0), p1);
-      } else if (op == GPUOS_OP_RMSNORM) {
-        float w[8];
-        ld8<DT>(E.in1, c, w);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) y[j] = __fmul_rn(__fmul_rn(x[j], p0), w[j]);
-      } else {
-        float g[8], b[8];
-        ld8<DT>(E.in1, c, g);
-        ld8<DT>(E.in2, c, b);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) y[j] = __fmaf_rn(__fmul_rn(x[j] - p0, p1), g[j], b[j]);
-      }
-      st8<DT>(E.out, rb + c, y);
-    }
+    out_span<DT, OP>(E, p0, p1, rb, c0, c1, lane);
   } else {
     // Unaligned row start. When the output (and the weights) sit at the same
     // offset modulo 16 bytes as the input row, the middle goes as ld8/st8.
@@ -727,14 +789,7 @@ static __device__ __noinline__ void row_out(const RingEntry& E, int, long long r
         const long long c = sp.cb + lane;
         st1<DT>(E.out, rb + c, row_apply1<DT>(E, op, p0, p1, ld1<DT>(E.in0, rb + c), c));
       }
-      for (long long c = sp.ca + (long long)lane * 8; c < sp.cb; c += 256) {
-        float x[8], w[8], b[8], y[8];
-        ld8<DT>(E.in0, rb + c, x);
-        if (op != GPUOS_OP_SOFTMAX) ld8<DT>(E.in1, c, w);
-        if (op == GPUOS_OP_LAYERNORM) ld8<DT>(E.in2, c, b);
-        row_apply8(op, p0, p1, x, w, b, y);
-        st8<DT>(E.out, rb + c, y);
-      }
+      out_span<DT, OP>(E, p0, p1, rb, sp.ca, sp.cb, lane);
     } else {
       // Element at a time, eight loads issued before the first store.
       long long c = c0 + lane;
@@ -1035,39 +1090,14 @@ static __device__ __noinline__ void row_item(const RingEntry& E, u32 item, u32 r
     const float K = (op == GPUOS_OP_LAYERNORM) ? ld1<DT>(E.in0, rb) : 0.f;
     Acc A = acc_init(op);
     if (vec) {
-      long long c = c0 + (long long)cx.lane * 8;
-      for (; c + (long long)(ROW_UNR - 1) * 256 < c1; c += (long long)ROW_UNR * 256) {
-        float x[ROW_UNR][8];
-#pragma unroll
-        for (int u = 0; u < ROW_UNR; ++u) ld8<DT>(E.in0, rb + c + u * 256, x[u]);
-#pragma unroll
-        for (int u = 0; u < ROW_UNR; ++u) acc8(op, A, x[u], K);
-      }
-      for (; c < c1; c += 256) {
-        float x[8];
-        ld8<DT>(E.in0, rb + c, x);
-        acc8(op, A, x, K);
-      }
+      acc_span<DT, ROW_UNR>(op, A, K, E.in0, rb, c0, c1, cx.lane);
     } else {
       // Row start not 16-byte aligned (ragged lengths): the lanes take the
       // few head and tail elements one each, the aligned middle as ld8.
       const RowSplit sp = row_split<DT>(E.in0, rb, c0, c1);
       if (cx.lane < sp.ca - c0) acc1(op, A, ld1<DT>(E.in0, rb + c0 + cx.lane), K);
       if (cx.lane < c1 - sp.cb) acc1(op, A, ld1<DT>(E.in0, rb + sp.cb + cx.lane), K);
-      long long c = sp.ca + (long long)cx.lane * 8;
-      constexpr int U = ROW_UNR / 2;
-      for (; c + (long long)(U - 1) * 256 < sp.cb; c += (long long)U * 256) {
-        float x[U][8];
-#pragma unroll
-        for (int u = 0; u < U; ++u) ld8<DT>(E.in0, rb + c + u * 256, x[u]);
-#pragma unroll
-        for (int u = 0; u < U; ++u) acc8(op, A, x[u], K);
-      }
-      for (; c < sp.cb; c += 256) {
-        float x[8];
-        ld8<DT>(E.in0, rb + c, x);
-        acc8(op, A, x, K);
-      }
+      acc_span<DT, ROW_UNR / 2>(op, A, K, E.in0, rb, sp.ca, sp.cb, cx.lane);
     }
     acc_warp(op, A);
     if (S == 1) {

@@ -677,7 +677,14 @@ __device__ void publisher(const KParams& p, Smem* S) {
         }
       }
       if (last) {
-        st_release_gpu(&p.done[idx], id + 1);
+        // A single-item op's outputs are covered by the batch fence above
+        // (fence + relaxed store is a release pattern). The last item of a
+        // large op acquired the other items' outputs through the counter,
+        // so its store itself must release them.
+        if (s.nitems > 1)
+          st_release_gpu(&p.done[idx], id + 1);
+        else
+          st_relaxed_gpu(&p.done[idx], id + 1);
         last_mask |= 1u << j;
       }
     }
@@ -747,7 +754,7 @@ constexpr size_t SMEM_HDR = (sizeof(Smem) + 127) / 128 * 128;
 constexpr size_t PERSISTENT_SMEM = SMEM_HDR + NCW * sizeof(WarpSmem);
 static_assert(PERSISTENT_SMEM <= 227 * 1024, "fits one SM");
 
-__global__ void __launch_bounds__(NTHREADS, 1) gpuos_persistent_kernel(const KParams p) {
+__global__ void __launch_bounds__(NTHREADS, 1) gpuos_persistent_kernel(const __grid_constant__ KParams p) {
   extern __shared__ __align__(128) unsigned char dsm[];
   Smem& S = *reinterpret_cast<Smem*>(dsm);
   WarpSmem* W = reinterpret_cast<WarpSmem*>(dsm + SMEM_HDR);
