@@ -137,6 +137,7 @@ typedef struct gpuos_config {
 #define GPUOS_CFG_NO_AUTOSTART 1u /* gpuos_create_ex does not launch the kernel */
 #define GPUOS_CFG_TRACE 2u        /* record a per-op event log (gpuos_trace_read) */
 #define GPUOS_CFG_NO_BULK 4u      /* op bodies read operands with plain loads only, no bulk-copy staging */
+#define GPUOS_CFG_NO_HANDOFF 8u   /* no chain hand-off: a claimed op always waits for its dependencies where it was claimed */
 
 #define GPUOS_START_DRAIN 1u      /* the kernel exits once every op published before gpuos_start completed */
 
@@ -164,7 +165,7 @@ typedef struct gpuos_trace_rec {
   uint32_t cta;     /* CTA that ran the last item */
   uint32_t smid;
   uint32_t items;   /* items run */
-  uint32_t claim;   /* 1 = claimed by chain affinity */
+  uint32_t claim;   /* how the op reached its CTA: 0 shared claim, 1 chain run, 2 large-op item, 3 chain hand-off */
 } gpuos_trace_rec;
 
 /* ---------------------------------------------------------------- lifecycle */

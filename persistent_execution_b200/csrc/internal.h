@@ -126,6 +126,18 @@ struct CtaStats {
 // baseline uses the same group size so both paths split rows identically.
 constexpr int NCW = 16;
 
+// Chain hand-off: a CTA that claims an op whose one unfinished dependency is
+// running on another CTA posts the op to that CTA's mailbox, and the owner
+// queues it right behind the dependency. owner[id & mask] = (id + 1) << 16 | cta
+// of the CTA that emitted single-item op id; mailboxes hold id + 1, 0 = empty.
+constexpr u32 MAILBOX = 16;
+struct MailCtl {
+  u64 tail;  // slots reserved by posting CTAs (CAS)
+  u64 pad0[7];
+  u64 head;  // slots taken by the owner
+  u64 pad1[7];
+};
+
 constexpr u32 KF_DRAIN = 1u;
 constexpr u32 KF_TRACE = 2u;
 constexpr u32 KF_NO_BULK = 4u;  // op bodies use register paths only (no bulk-copy staging)
@@ -140,6 +152,9 @@ struct KParams {
   u64* hdone;              // device alias of the host completion array
   CtaStats* stats;
   gpuos_trace_rec* trace;
+  u64* owner;     // [capacity], or null: no chain hand-off
+  u64* mbox;      // [grid * MAILBOX]
+  MailCtl* mctl;  // [grid]
   u64 mask;  // capacity - 1
   u64 base;  // first id of the session
   u64 timeout_ns;

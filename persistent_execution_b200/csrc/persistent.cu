@@ -46,7 +46,7 @@ constexpr unsigned LOOKAHEAD = 2;
 constexpr unsigned FULLMASK = 0xffffffffu;
 
 enum : u32 { SLOT_WORK = 0, SLOT_EXIT = 1 };
-enum : u32 { CLAIM_SHARED = 0, CLAIM_RUN = 1, CLAIM_BIG = 2 };
+enum : u32 { CLAIM_SHARED = 0, CLAIM_RUN = 1, CLAIM_BIG = 2, CLAIM_MAIL = 3 };
 
 struct __align__(16) Slot {
   RingEntry e;
@@ -65,8 +65,10 @@ struct Smem {
   u64 free_bar[FIFO];
   float4 part[NCW];
   u64 recent[8];
+  u64 deferred[32];         // mailbox ops waiting for the op this CTA holds (ids)
   volatile unsigned ncomp;  // items the compute warps finished
 };
+constexpr u32 DEFER = 32;
 
 __device__ __forceinline__ u64 bcast(u64 v) { return __shfl_sync(FULLMASK, v, 0); }
 __device__ __forceinline__ u32 bcast32(u32 v) { return __shfl_sync(FULLMASK, v, 0); }
@@ -88,6 +90,9 @@ struct Control {
   u32 backoff = 0;
   u32 iters = 0;
   u64 claimed = 0, runops = 0, idle_cyc = 0, dep_cyc = 0, fetched = 0;
+  u64 mb_head = 0;                // mailbox slots this CTA has taken
+  u64 held = 0;                   // id + 1 of the single op claimed here and not yet emitted
+  u32 ndef = 0;                   // entries of S->deferred
   const bool drain;
 
   __device__ Control(const KParams& pp, Smem* s, int l) : p(pp), S(s), lane(l), drain((pp.flags & KF_DRAIN) != 0) {}
@@ -116,72 +121,190 @@ struct Control {
     nrecent = nrecent + 1 > 8 ? 8 : nrecent + 1;
   }
 
-  // Waits until the op encoded as d (id + 1, 0 = none) completed. False on abort/timeout.
-  __device__ __forceinline__ bool wait_dep(u64 d, u64 id) {
-    if (d == 0) return true;
-    const u64 dd = d - 1;
-    if (is_local(dd)) return true;
-    u32 ok = 0;
-    if (lane == 0) {
-      const u64 c0 = clock64();
-      const u64 t0 = globaltimer();
-      const u64* w = &p.done[dd & p.mask];
-      for (u32 spins = 0;; ++spins) {
-        if (ld_acquire_gpu(w) >= d) {
-          ok = 1;
+  // Mailbox slot this CTA reads next.
+  __device__ __forceinline__ u64* mail_slot() const { return &p.mbox[(u64)blockIdx.x * MAILBOX + (mb_head % MAILBOX)]; }
+  __device__ __forceinline__ bool mail_ready() const { return p.mbox && ld_acquire_gpu(mail_slot()) != 0; }
+
+  // Lane 0: polls the completion words of d0, d1 (id + 1, 0 = none) and the
+  // mailbox. 1 = both done, 2 = an op arrived in the mailbox, 0 = abort or
+  // timeout (timed from t0).
+  __device__ __forceinline__ u32 spin_deps(u64 id, u64 d0, u64 d1, u64 t0, bool mail = true) {
+    const u64* w0 = d0 ? &p.done[(d0 - 1) & p.mask] : nullptr;
+    const u64* w1 = d1 ? &p.done[(d1 - 1) & p.mask] : nullptr;
+    const u64 c0 = clock64();
+    u32 r = 0;
+    for (u32 spins = 0;; ++spins) {
+      const bool ok0 = !w0 || ld_acquire_gpu(w0) >= d0;
+      const bool ok1 = !w1 || ld_acquire_gpu(w1) >= d1;
+      if (ok0 && ok1) {
+        r = 1;
+        break;
+      }
+      if (mail && mail_ready()) {
+        r = 2;
+        break;
+      }
+      if ((spins & 63) == 63) {
+        if (aborted()) break;
+        if (globaltimer() - t0 > p.timeout_ns) {
+          raise_error(p.st, p.hctl, GPUOS_ETIMEDOUT, id);
           break;
         }
-        if ((spins & 63) == 63) {
-          if (aborted()) break;
-          if (globaltimer() - t0 > p.timeout_ns) {
-            raise_error(p.st, p.hctl, GPUOS_ETIMEDOUT, id);
-            break;
-          }
-        }
-        if (spins > 64) __nanosleep(spins > 4096 ? 256 : 32);
       }
-      dep_cyc += clock64() - c0;
+      if (spins > 64) __nanosleep(spins > 4096 ? 256 : 32);
     }
-    return bcast32(ok) != 0;
+    dep_cyc += clock64() - c0;
+    return r;
   }
 
-  // Both dependencies, polled together (one L2 round trip when both are done).
+  // Waits until both dependencies (id + 1, 0 = none) of op id completed; ops
+  // that arrive in the mailbox meanwhile are queued first (one of them may be
+  // what id waits for). False on abort or timeout.
   __device__ __forceinline__ bool wait_deps(u64 id, u64 d0, u64 d1) {
     if (d0 != 0 && is_local(d0 - 1)) d0 = 0;
     if (d1 != 0 && is_local(d1 - 1)) d1 = 0;
-    if (d0 == 0 || d1 == 0) return wait_dep(d0 | d1, id);
+    if ((d0 | d1) == 0) return true;
+    const u64 t0 = lane == 0 ? globaltimer() : 0ull;
+    bool mail = true;
+    for (;;) {
+      u32 r = 0;
+      if (lane == 0) r = spin_deps(id, d0, d1, t0, mail);
+      r = bcast32(r);
+      if (r == 1) return true;
+      if (r == 0) return false;
+      const int m = serve_mail(false);
+      if (m < 0) return false;
+      if (m == 0) mail = false;  // nothing could be taken (deferred list full): wait without the mailbox
+    }
+  }
+
+  __device__ __forceinline__ void set_owner(u64 c) {
+    if (p.owner && lane == 0) st_relaxed_gpu(&p.owner[c & p.mask], ((c + 1) << 16) | (u64)blockIdx.x);
+  }
+
+  // Queues a mailbox op: emitted, owned here from now on.
+  __device__ __forceinline__ bool emit_mail(u64 c) {
+    if (!emit(c, 0, 1, CLAIM_MAIL)) return false;
+    note_single(c);
+    set_owner(c);
+    return true;
+  }
+
+  // Takes the next op from this CTA's mailbox, if any. The poster saw every
+  // dependency but one complete, and that one owned here: emitted (the op
+  // then runs after it in FIFO order) or held (the op is deferred until the
+  // held op is emitted). -1 error, 0 empty, 1 taken.
+  // extend: also claim the FOLLOW ops after it as a run (only where no run or
+  // claimed op is in progress).
+  __device__ __forceinline__ int serve_mail(bool extend) {
+    if (!p.mbox || ndef >= DEFER) return 0;
+    u64 v = 0, d0 = 0, d1 = 0;
+    if (lane == 0) {
+      u64* slot = mail_slot();
+      v = ld_acquire_gpu(slot);
+      if (v != 0) {
+        st_relaxed_gpu(slot, 0ull);
+        st_release_gpu(&p.mctl[blockIdx.x].head, mb_head + 1);  // the slot is free again
+        d0 = ent(v - 1)->dep0;
+        d1 = ent(v - 1)->dep1;
+      }
+    }
+    v = bcast(v);
+    if (v == 0) return 0;
+    ++mb_head;
+    const u64 c = v - 1;
+    d0 = bcast(d0);
+    d1 = bcast(d1);
+    if (held != 0 && (waits_held(d0) || waits_held(d1))) {
+      if (lane == 0) S->deferred[ndef] = c;
+      __syncwarp();
+      ++ndef;
+      return 1;
+    }
+    // the dependency is local or done; anything else is waited for here
+    if (d0 != 0 && is_local(d0 - 1)) d0 = 0;
+    if (d1 != 0 && is_local(d1 - 1)) d1 = 0;
+    if ((d0 | d1) != 0) {
+      u32 r = 0;
+      if (lane == 0) r = spin_deps(c, d0, d1, globaltimer(), false);
+      if (bcast32(r) != 1) return -1;
+    }
+    if (!emit_mail(c)) return -1;
+    if (extend && run_next >= run_end) try_extend(c);
+    return 1;
+  }
+
+  // True if d (id + 1) is the held op or a mailbox op deferred behind it.
+  __device__ __forceinline__ bool waits_held(u64 d) {
+    if (d == 0) return false;
+    if (d == held) return true;
+    const bool hit = (u32)lane < ndef && S->deferred[lane] + 1 == d;
+    return __any_sync(FULLMASK, hit);
+  }
+
+  // After the held op is emitted: the mailbox ops that waited for it.
+  __device__ __forceinline__ bool release_held() {
+    held = 0;
+    for (u32 i = 0; i < ndef; ++i) {
+      u64 c = 0;
+      if (lane == 0) c = S->deferred[i];
+      if (!emit_mail(bcast(c))) return false;
+    }
+    ndef = 0;
+    return true;
+  }
+
+  // Posts single-item op c, whose dependencies are d0, d1 (id + 1, 0 = none),
+  // to the CTA that emitted its one unfinished dependency. True if posted;
+  // false leaves c to the caller (nothing to wait for, two unfinished
+  // dependencies, an unknown or local owner, or a full mailbox).
+  __device__ __forceinline__ bool try_handoff(u64 c, u64 d0, u64 d1) {
+    if (!p.mbox || (d0 | d1) == 0) return false;
+    if ((d0 != 0 && is_local(d0 - 1)) || (d1 != 0 && is_local(d1 - 1))) return false;
     u32 ok = 0;
     if (lane == 0) {
-      const u64 c0 = clock64();
-      const u64 t0 = globaltimer();
-      const u64* w0 = &p.done[(d0 - 1) & p.mask];
-      const u64* w1 = &p.done[(d1 - 1) & p.mask];
-      for (u32 spins = 0;; ++spins) {
-        const u64 v0 = ld_acquire_gpu(w0), v1 = ld_acquire_gpu(w1);
-        if (v0 >= d0 && v1 >= d1) {
-          ok = 1;
-          break;
-        }
-        if ((spins & 63) == 63) {
-          if (aborted()) break;
-          if (globaltimer() - t0 > p.timeout_ns) {
-            raise_error(p.st, p.hctl, GPUOS_ETIMEDOUT, id);
-            break;
+      const bool u0 = d0 != 0 && ld_acquire_gpu(&p.done[(d0 - 1) & p.mask]) < d0;
+      const bool u1 = d1 != 0 && ld_acquire_gpu(&p.done[(d1 - 1) & p.mask]) < d1;
+      if (u0 != u1) {
+        const u64 a = u0 ? d0 : d1;
+        const u64 o = ld_relaxed_gpu(&p.owner[(a - 1) & p.mask]);
+        const u32 cta = (u32)(o & 0xffffu);
+        if ((o >> 16) == a && cta != blockIdx.x && cta < p.grid) {
+          MailCtl* m = &p.mctl[cta];
+          const u64 t = ld_relaxed_gpu(&m->tail);
+          const u64 h = ld_acquire_gpu(&m->head);
+          if (t - h < MAILBOX && atomicCAS(&m->tail, t, t + 1) == t) {
+            st_release_gpu(&p.mbox[(u64)cta * MAILBOX + (t % MAILBOX)], c + 1);
+            // c is owned there from now on: its own dependants follow it
+            st_relaxed_gpu(&p.owner[c & p.mask], ((c + 1) << 16) | (u64)cta);
+            ok = 1;
           }
         }
-        if (spins > 64) __nanosleep(spins > 4096 ? 256 : 32);
       }
-      dep_cyc += clock64() - c0;
     }
     return bcast32(ok) != 0;
   }
 
   // Waits until this CTA has fewer than `lim` items emitted but not finished.
-  __device__ __forceinline__ void throttle(unsigned lim) {
-    if (lane == 0) {
-      while ((unsigned)k - S->ncomp >= lim) __nanosleep(20);
+  // Mailbox ops that arrive meanwhile are queued at once. False on error.
+  __device__ __forceinline__ bool throttle(unsigned lim) {
+    bool mail = p.mbox != nullptr;
+    for (;;) {
+      u32 r = 0;
+      if (lane == 0) {
+        for (u32 spins = 0; (unsigned)k - S->ncomp >= lim; ++spins) {
+          if (mail && (spins & 15) == 15 && mail_ready()) {  // a global load: not on every spin
+            r = 1;
+            break;
+          }
+          __nanosleep(20);
+        }
+      }
+      if (bcast32(r) == 0) return true;
+      const int m = serve_mail(true);
+      if (m < 0) return false;
+      if (m == 0) mail = false;
     }
-    __syncwarp();
   }
 
   // Copies one entry into the next FIFO slot and signals the compute warps.
@@ -303,6 +426,8 @@ struct Control {
 
   // Nothing claimable: poll, fetch, decide exit, back off. False = leave.
   __device__ __forceinline__ bool idle_step() {
+    const int m = serve_mail(false);
+    if (m != 0) return m > 0;
     const u64 c0 = clock64();
     u32 leave = 0;
     if (lane == 0) {
@@ -384,7 +509,9 @@ struct Control {
     }
   }
 
-  __device__ __forceinline__ bool emit_single(u64 c, u32 claim, const RingEntry* staged = nullptr) {
+  // 0 error, 1 emitted here, 2 posted to the CTA running its unfinished dependency.
+  __device__ __forceinline__ int emit_single(u64 c, u32 claim, const RingEntry* staged = nullptr,
+                                             bool handoff = false) {
     u64 d0 = 0, d1 = 0;
     if (lane == 0) {
       const RingEntry* e = staged ? staged : ent(c);
@@ -393,10 +520,17 @@ struct Control {
     }
     d0 = bcast(d0);
     d1 = bcast(d1);
-    if (!wait_deps(c, d0, d1)) return false;
-    if (!emit(c, 0, 1, claim, staged)) return false;
+    if (handoff) {
+      if (try_handoff(c, d0, d1)) return 2;
+      held = c + 1;  // dependants may be posted here from now on
+      set_owner(c);
+    }
+    if (!wait_deps(c, d0, d1)) return 0;
+    if (!emit(c, 0, 1, claim, staged)) return 0;
     note_single(c);
-    return true;
+    set_owner(c);
+    if (handoff && !release_held()) return 0;
+    return 1;
   }
 
   // -1 error, 0 nothing to join, 1 emitted an item of the open large op.
@@ -541,8 +675,9 @@ struct Control {
         pend_word = ~0ull;
         return 1;
       }
-      if (!emit_single(c2, CLAIM_SHARED)) return -1;
-      try_extend(c2);
+      const int r = emit_single(c2, CLAIM_SHARED, nullptr, true);
+      if (r == 0) return -1;
+      if (r == 1) try_extend(c2);
       return 1;
     }
     if (hdr_items(h) > 1) {
@@ -553,9 +688,13 @@ struct Control {
     // dependencies straight from the entry in registers (dep0: lane 0, dep1: lane 1)
     const u64 d0 = __shfl_sync(FULLMASK, (u64)chunk.z | ((u64)chunk.w << 32), 0);
     const u64 d1 = __shfl_sync(FULLMASK, (u64)chunk.x | ((u64)chunk.y << 32), 1);
+    if (try_handoff(c, d0, d1)) return 1;
+    held = c + 1;  // dependants may be posted here from now on
+    set_owner(c);
     if (!wait_deps(c, d0, d1)) return -1;
     if (!emit(c, 0, 1, CLAIM_SHARED, nullptr, true, chunk)) return -1;
     note_single(c);
+    if (!release_held()) return -1;
     try_extend(c);
     return 1;
   }
@@ -572,7 +711,12 @@ struct Control {
         backoff = 0;
         continue;
       }
-      throttle(LOOKAHEAD);
+      {
+        const int m = serve_mail(true);
+        if (m < 0) break;
+        if (m > 0) continue;
+      }
+      if (!throttle(LOOKAHEAD)) break;
       if (pending) {
         const int r = try_install(pending - 1);
         if (r < 0) break;
@@ -819,7 +963,13 @@ __global__ void gpuos_reset_kernel(const KParams p, u64 head, u64 big_init) {
   for (u64 i = tid; i < p.grid; i += nth) {
     CtaStats z = {};
     p.stats[i] = z;
+    if (p.mctl) {
+      p.mctl[i].tail = 0;
+      p.mctl[i].head = 0;
+    }
   }
+  if (p.mbox)
+    for (u64 i = tid; i < (u64)p.grid * MAILBOX; i += nth) p.mbox[i] = 0;
 }
 
 int launch_session(const KParams& p, u64 head, u64 big_init, void* stream) {

@@ -144,6 +144,9 @@ struct gpuos {
   RingEntry* dring = nullptr;
   u64* done = nullptr;
   u32* tiles_done = nullptr;
+  u64* owner = nullptr;
+  u64* mbox = nullptr;
+  MailCtl* mctl = nullptr;
   CtaStats* cstats = nullptr;
   gpuos_trace_rec* trace = nullptr;
   u64 cap = 0, mask = 0;
@@ -245,6 +248,10 @@ gpuos_status start_kernel(gpuos* rt, u32 flags) {
   p.hdone = rt->hdone_d;
   p.stats = rt->cstats;
   p.trace = rt->trace;
+  const bool handoff = !(rt->cfg.flags & GPUOS_CFG_NO_HANDOFF);
+  p.owner = handoff ? rt->owner : nullptr;
+  p.mbox = handoff ? rt->mbox : nullptr;
+  p.mctl = handoff ? rt->mctl : nullptr;
   p.mask = rt->mask;
   p.base = base;
   p.timeout_ns = rt->cfg.timeout_ns;
@@ -417,6 +424,9 @@ void free_all(gpuos* rt) {
   if (rt->dring) cudaFree(rt->dring);
   if (rt->done) cudaFree(rt->done);
   if (rt->tiles_done) cudaFree(rt->tiles_done);
+  if (rt->owner) cudaFree(rt->owner);
+  if (rt->mbox) cudaFree(rt->mbox);
+  if (rt->mctl) cudaFree(rt->mctl);
   if (rt->cstats) cudaFree(rt->cstats);
   if (rt->trace) cudaFree(rt->trace);
   if (rt->aux) cudaStreamDestroy(rt->aux);
@@ -480,6 +490,9 @@ gpuos_status gpuos_create_ex(gpuos_stream_t stream, const gpuos_config* cfg_in, 
   ok = ok && cudaMalloc((void**)&rt->done, rt->cap * sizeof(u64)) == cudaSuccess;
   ok = ok && cudaMalloc((void**)&rt->tiles_done, rt->cap * sizeof(u32)) == cudaSuccess;
   ok = ok && cudaMalloc((void**)&rt->cstats, rt->grid * sizeof(CtaStats)) == cudaSuccess;
+  ok = ok && cudaMalloc((void**)&rt->owner, rt->cap * sizeof(u64)) == cudaSuccess;
+  ok = ok && cudaMalloc((void**)&rt->mbox, (size_t)rt->grid * MAILBOX * sizeof(u64)) == cudaSuccess;
+  ok = ok && cudaMalloc((void**)&rt->mctl, rt->grid * sizeof(MailCtl)) == cudaSuccess;
   if (ok && (cfg.flags & GPUOS_CFG_TRACE))
     ok = cudaMalloc((void**)&rt->trace, rt->cap * sizeof(gpuos_trace_rec)) == cudaSuccess;
   ok = ok && cudaMemsetAsync(rt->st, 0, sizeof(DevState), rt->aux) == cudaSuccess;
@@ -487,6 +500,7 @@ gpuos_status gpuos_create_ex(gpuos_stream_t stream, const gpuos_config* cfg_in, 
   ok = ok && cudaMemsetAsync(rt->done, 0, rt->cap * sizeof(u64), rt->aux) == cudaSuccess;
   ok = ok && cudaMemsetAsync(rt->tiles_done, 0, rt->cap * sizeof(u32), rt->aux) == cudaSuccess;
   ok = ok && cudaMemsetAsync(rt->cstats, 0, rt->grid * sizeof(CtaStats), rt->aux) == cudaSuccess;
+  ok = ok && cudaMemsetAsync(rt->owner, 0, rt->cap * sizeof(u64), rt->aux) == cudaSuccess;
   ok = ok && cudaStreamSynchronize(rt->aux) == cudaSuccess;
   if (!ok) {
     cudaGetLastError();

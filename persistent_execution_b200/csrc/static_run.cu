@@ -158,6 +158,9 @@ extern "C" gpuos_status gpuos_run_static(const gpuos_desc* descs, uint64_t n, co
   p.hdone = reinterpret_cast<u64*>(base + OFF_HDONE);
   p.stats = reinterpret_cast<CtaStats*>(base + OFF_STATS);
   p.trace = nullptr;
+  p.owner = nullptr;  // no chain hand-off: the array holds no mailboxes
+  p.mbox = nullptr;
+  p.mctl = nullptr;
   p.mask = STATIC_MAX_OPS - 1;
   p.base = 0;
   p.timeout_ns = cfg.timeout_ns;

@@ -124,6 +124,25 @@ def test_chain_affinity_keeps_chains_on_one_cta():
     assert len(np.unique(tr["cta"])) <= 3
 
 
+@pytest.mark.parametrize("mode", ["drain", "live"])
+def test_chain_handoff_interleaved_streams(mode):
+    # config 4's request chains are interleaved, so a claimed op's predecessor
+    # usually runs on another CTA: the claimer posts it to that CTA's mailbox.
+    w = W.make(4, small=True)
+    a32, a16, tr, st = U.run_persistent(w, mode=mode, trace=True, batch=101)
+    assert not P.check_ops(w, a32, a16)
+    assert T.violations(w.ops["dep"], tr["t_start"], tr["t_end"]) == []
+    handed = tr["claim"] == 3
+    assert handed.any(), np.bincount(tr["claim"])
+    # a handed-off op runs on the CTA that ran its predecessor
+    dep = w.ops["dep"][:, 0]
+    idx = np.nonzero(handed & (dep >= 0))[0]
+    assert (tr["cta"][idx] == tr["cta"][dep[idx]]).mean() > 0.99
+    # the same stream without hand-off gives bit-identical outputs
+    b32, b16, _, _ = U.run_persistent(w, mode=mode, cfg=dict(flags=G.CFG_NO_HANDOFF), batch=101)
+    assert P.bit_exact(w, a32, a16, b32, b16) == []
+
+
 @pytest.mark.parametrize("config", [2, 4])
 def test_baselines_match_persistent(config):
     w = W.make(config, small=True)
