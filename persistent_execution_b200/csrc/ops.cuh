@@ -178,6 +178,24 @@ static __device__ __noinline__ float gelu_f(float x) {
   double xd = (double)x;
   return (float)(0.5 * xd * erfc(-xd / 1.4142135623730951));
 }
+// gelu of the standalone fp32 op: 0.5 x erfc(t) at t = -x/sqrt(2), with t
+// carried as a float plus its rounding error dt (the exact product error by
+// fma, and the low part of 1/sqrt(2)), and erfc corrected to first order,
+// erfc(t + dt) = erfc(t) - (2/sqrt(pi)) exp(-t^2) dt. Without dt the relative
+// error of erfc would grow like 2 t^2 2^-24 (1e-6 at |x| = 4.2); with it the
+// error is that of erfcf (4 ulp by CUDA's documentation) plus two roundings,
+// under 1e-6 relative. Tails (|x| > 10, where erfc nears the subnormal range),
+// tiny and non-finite x take the double path.
+__device__ __forceinline__ float gelu_fast(float x) {
+  const float ax = fabsf(x);
+  if (!(ax <= 10.0f) || ax < 1e-30f) return gelu_f(x);
+  const float c_hi = 0.70710677f, c_lo = 1.2101617e-08f;  // 1/sqrt(2) = c_hi + c_lo
+  const float nx = -x;
+  const float t = __fmul_rn(nx, c_hi);
+  const float dt = __fadd_rn(__fmaf_rn(nx, c_hi, -t), __fmul_rn(nx, c_lo));
+  const float r = erfcf(t) - 1.1283791671f * __expf(-t * t) * dt;
+  return 0.5f * x * r;
+}
 static __device__ __noinline__ float silu_f(float x) {
   double xd = (double)x;
   return (float)(xd / (1.0 + exp(-xd)));
@@ -232,7 +250,7 @@ __device__ __forceinline__ float ew_f(const RingEntry& E, float x0, float x1, fl
   if (OPK == GPUOS_OP_ADD) return __fadd_rn(x0, x1);
   if (OPK == GPUOS_OP_MUL) return __fmul_rn(x0, x1);
   if (OPK == GPUOS_OP_SCALE) return __fmul_rn(E.s[0], x0);
-  if (OPK == GPUOS_OP_GELU) return gelu_f(x0);
+  if (OPK == GPUOS_OP_GELU) return gelu_fast(x0);
   if (OPK == GPUOS_OP_RELU_AFFINE) return relu_f(__fmaf_rn(E.s[0], x0, E.s[1]));
   if (OPK == GPUOS_OP_SILU_MUL) return DT == 1 ? silu_mul_bf(x0, x1) : silu_mul_f(x0, x1);
   return chain_f(E, x0, x1, x2);  // GPUOS_OP_EW_CHAIN, OPK_CHAIN_CALLS

@@ -376,7 +376,14 @@ struct Control {
     if (lane == 0) {
       fn = ld_relaxed_gpu(&p.st->fetch_next.v);
       const u64 hm = ld_acquire_gpu(&p.st->head_mirror.v);
-      if (fn < hm) {
+      if (drain && fn < hm) {
+        // drained session: the head is fixed, so every CTA takes its own
+        // batch at once; a batch that starts at or past the head is empty
+        fn = atomicAdd(&p.st->fetch_next.v, 32ull);
+        e = fn + 32 < hm ? fn + 32 : hm;
+        got = fn < hm;
+        if (!got) e = fn;
+      } else if (fn < hm) {
         e = fn + 32 < hm ? fn + 32 : hm;
         got = atomicCAS(&p.st->fetch_next.v, fn, e) == fn;
         if (!got) e = fn + 1;  // someone else took it: still progress

@@ -63,6 +63,15 @@ def test_elementwise_broadcast(dtype):
             assert not f and not fb, (kind, n, n0, n1, f, fb)
 
 
+@pytest.mark.parametrize("sd", [1.0, 4.0, 12.0])
+def test_gelu_fp32_wide_range(sd):
+    # the fp32 gelu path over the bulk (|x| <= 10) and the double-precision
+    # tails, within 1e-6 relative of the oracle element by element
+    w = W.single_op("gelu", 0, 1, 1 << 20, seed=int(sd * 10), sd=sd)
+    _, _, _, _, f, fb = _run_both(w)
+    assert not f and not fb, (f, fb)
+
+
 ROW_SHAPES = [(1, 1), (3, 5), (7, 1000), (16, 1024), (1, 2048), (8, 4096), (5, 4100), (2000, 64),
               (3, 8192), (9, 65536 + 8)]
 
@@ -150,6 +159,22 @@ def test_baselines_match_persistent(config):
     for mode in (None, 0, 1):
         b32, b16 = U.run_launches(w, graph_mode=mode)
         assert P.bit_exact(w, a32, a16, b32, b16) == [], mode
+
+
+@pytest.mark.parametrize("mode", ["drain", "live"])
+def test_long_dag_with_multi_item_ops(mode):
+    # a long DAG stream with 1024-element items: most ops are multi-item
+    # (opened in submission order, joined by many CTAs) between single-item ones
+    w = W.make(2, n_ops=6000)
+    a32, a16, tr, st = U.run_persistent(w, mode=mode, trace=True, batch=1500,
+                                        cfg={"elem_chunk": 1024, "ring_capacity": 8192})
+    assert not P.check_ops(w, a32, a16)
+    assert T.violations(w.ops["dep"], tr["t_start"], tr["t_end"]) == []
+    d = streams.descriptors(w, 1 << 20, 1 << 21)
+    c = G.default_config(elem_chunk=1024)
+    items = np.array([G.gpuos_work_items(d[i:i + 1], c) for i in range(w.n_ops)])
+    assert (tr["items"] == items).all()
+    assert (items > 1).mean() > 0.3
 
 
 def test_large_multi_item_ops_and_chunk_sizes():
