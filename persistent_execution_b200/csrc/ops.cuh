@@ -184,11 +184,13 @@ static __device__ __noinline__ float gelu_f(float x) {
 // erfc(t + dt) = erfc(t) - (2/sqrt(pi)) exp(-t^2) dt. Without dt the relative
 // error of erfc would grow like 2 t^2 2^-24 (1e-6 at |x| = 4.2); with it the
 // error is that of erfcf (4 ulp by CUDA's documentation) plus two roundings,
-// under 1e-6 relative. Tails (|x| > 10, where erfc nears the subnormal range),
-// tiny and non-finite x take the double path.
+// under 1e-6 relative. For x >= 6, Phi(x) > 1 - 2^-26 and x Phi(x) rounds
+// to x; for |x| < 1e-30, Phi(x) = 1/2 far below an ulp; x < -10 (where the
+// result nears the subnormal range), -inf and NaN take the double path.
 __device__ __forceinline__ float gelu_fast(float x) {
-  const float ax = fabsf(x);
-  if (!(ax <= 10.0f) || ax < 1e-30f) return gelu_f(x);
+  if (x >= 6.0f) return x;
+  if (fabsf(x) < 1e-30f) return 0.5f * x;
+  if (!(x >= -10.0f)) return gelu_f(x);
   const float c_hi = 0.70710677f, c_lo = 1.2101617e-08f;  // 1/sqrt(2) = c_hi + c_lo
   const float nx = -x;
   const float t = __fmul_rn(nx, c_hi);
