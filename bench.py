@@ -140,15 +140,9 @@ class Clocks:
 
 
 def setup_dist(args):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import torch.distributed as dist
-        backend = "gloo" if args.impl == "reference" else "nccl"
-        import datetime
-        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
-    return rank, world, local
+    from persistent_execution_b200 import replicas as R
+    r = R.init("gloo" if args.impl == "reference" else "nccl")
+    return r.rank, r.world, r.local
 
 
 # ---------------------------------------------------------------- reference arm (CPU oracle)
@@ -208,6 +202,7 @@ def bench_gpu(args, rank, world, local):
     from persistent_execution_b200 import build as B
     from persistent_execution_b200 import gpuos as G
     from persistent_execution_b200 import measure as Ms
+    from persistent_execution_b200 import replicas as R
     from persistent_execution_b200 import streams
     from persistent_execution_b200 import workloads as W
 
@@ -270,9 +265,8 @@ def bench_gpu(args, rank, world, local):
     first_of = [rt.submit_n(descs, dep_base=0)]
     rt.flush()
     torch.cuda.synchronize()
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    ranks = R.from_env()
+    R.barrier(ranks)
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     st0 = rt.stats()
@@ -281,20 +275,15 @@ def bench_gpu(args, rank, world, local):
         step_loop(args.steps, ev)
         torch.cuda.synchronize()
     t_wall = time.perf_counter() - t_wall
-    if world > 1:
-        dist.barrier()
+    R.barrier(ranks)
     torch.cuda.synchronize()
     st1 = rt.stats()
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    elapsed_ms = float(np.sum(step_ms))
-    if world > 1:
-        t = torch.tensor([elapsed_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = R.max_over_ranks(ranks, float(np.sum(step_ms)), device="cuda")
     launches = st1["kernel_launches"] - st0["kernel_launches"]
     span_ns = st1["gpu_span_ns"]
     ms_step = elapsed_ms / args.steps
-    value = world * n * args.steps / (elapsed_ms / 1e3)
+    value = R.job_throughput(n * args.steps, ranks, elapsed_ms / 1e3)
     per_launch_s = float(np.mean(step_ms)) / 1e3  # one persistent kernel (and its reset kernel) per step
     peak, peak_kind = measured_peak()
     achieved = alg_bytes / per_launch_s / 1e9
@@ -335,8 +324,8 @@ def bench_gpu(args, rank, world, local):
             G.check(rt.stop(120.0), "e2e stop")
             if rep > 0:
                 tms.append(e0.elapsed_time(e1))
-        e2e_ms = float(np.median(tms))
-        e2e = {"value": world * n / (e2e_ms / 1e3), "unit": "ops/s", "h2d_bytes_per_step": int(h2d),
+        e2e_ms = R.max_over_ranks(ranks, float(np.median(tms)), device="cuda")
+        e2e = {"value": R.job_throughput(n, ranks, e2e_ms / 1e3), "unit": "ops/s", "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms}
 
     baselines = None
@@ -438,9 +427,8 @@ def main():
         else:
             bench_gpu(args, rank, world, local)
     finally:
-        if world > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
+        from persistent_execution_b200 import replicas as R
+        R.finalize(R.from_env())
 
 
 if __name__ == "__main__":
