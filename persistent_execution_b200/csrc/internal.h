@@ -157,6 +157,7 @@ struct KParams {
   MailCtl* mctl;  // [grid]
   u64 mask;  // capacity - 1
   u64 base;  // first id of the session
+  u64 fetched_upto;  // ids in [base, fetched_upto) are already in the device ring
   u64 timeout_ns;
   u64 idle_exit_ns;
   u32 elem_chunk, row_chunk, backoff_ns, flags, grid;

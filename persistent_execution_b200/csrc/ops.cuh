@@ -545,7 +545,10 @@ __device__ __forceinline__ bool chain_calls(const RingEntry& E) {
 template <int DT>
 __device__ void ew_item(const RingEntry& E, u32 item, u32 elem_chunk, const Cx& cx) {
   const long long n = E.rows * E.cols;
-  const bool s0 = E.in_n0 == n && al16(E.in0) && !(cx.flags & KF_NO_BULK);
+  // Bulk-copy staging pays off when the whole grid streams one large op from
+  // HBM (an op of several items); a single-item op is latency-bound on one SM,
+  // where the register path's loads arrive sooner.
+  const bool s0 = E.in_n0 == n && al16(E.in0) && !(cx.flags & KF_NO_BULK) && n > (long long)elem_chunk;
   const bool s1 = E.in_n1 == n && al16(E.in1);
   if (s0 && al16(E.out)) {
     bool u1 = false, u2 = false;

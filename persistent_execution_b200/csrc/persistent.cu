@@ -940,7 +940,7 @@ __global__ void gpuos_reset_kernel(const KParams p, u64 head, u64 big_init) {
   if (tid == 0) {
     DevState* st = p.st;
     st->next_op.v = p.base;
-    st->fetch_next.v = p.base;
+    st->fetch_next.v = p.fetched_upto > p.base ? p.fetched_upto : p.base;
     st->head_mirror.v = head;
     st->big.v = big_init;
     st->poll_lock.v = 0;

@@ -5,14 +5,15 @@
 // next dense id, build its 128-byte ring entry and write it into the pinned,
 // write-combined, device-mapped ring. Flush is a store fence plus one store of
 // the head counter into mapped memory -- the user-space counterpart of the
-// driver's "pinned ring buffer in host memory" and doorbell ("Kernel Launch
-// and Host-Device Interaction", section 5, "The launch path", steps 3-4).
+// driver's pinned host ring and doorbell ("Kernel Launch and Host-Device
+// Interaction", section 5, "The launch path").
 // Waiting reads the per-op completion entries the device writes into mapped
 // memory, so there is no implicit synchronisation per op (same page,
 // "Synchronization primitives").
 #include <cuda_runtime.h>
 #include <immintrin.h>
 
+#include <algorithm>
 #include <chrono>
 #include <cstring>
 #include <deque>
@@ -151,6 +152,8 @@ struct gpuos {
   gpuos_trace_rec* trace = nullptr;
   u64 cap = 0, mask = 0;
   u64 next_id = 0, published = 0, tail = 0, session_base = 0;
+  u64 dma_upto = 0;               // ids below this were copied into the device ring by the copy engine
+  cudaEvent_t dma_ev = nullptr;   // the last such copy
   bool running = false;
   bool kernel_alive = false;  // false only if a kernel could not be confirmed stopped
   u32 run_flags = 0;
@@ -228,6 +231,23 @@ void retire_bigs(gpuos* rt, u64 upto) {
   }
 }
 
+// Copies the host entries of ids [from, to) into their device-ring slots with
+// the copy engine (aux stream). A drained session then starts with its whole
+// stream in device memory: its CTAs do not read descriptors over PCIe while
+// ops run, which would hold up the loads of the running ops on every SM.
+bool dma_ring(gpuos* rt, u64 from, u64 to) {
+  while (from < to) {
+    const u64 s = from & rt->mask;
+    const u64 m = std::min(to - from, rt->cap - s);
+    if (cudaMemcpyAsync(rt->dring + s, rt->hring + s, m * sizeof(RingEntry), cudaMemcpyHostToDevice, rt->aux) !=
+        cudaSuccess)
+      return false;
+    from += m;
+  }
+  rt->dma_upto = to;
+  return cudaEventRecord(rt->dma_ev, rt->aux) == cudaSuccess;
+}
+
 gpuos_status start_kernel(gpuos* rt, u32 flags) {
   if (rt->sticky != GPUOS_OK) return rt->sticky;
   if (rt->running) return GPUOS_EINVAL;
@@ -262,6 +282,20 @@ gpuos_status start_kernel(gpuos* rt, u32 flags) {
   p.flags = ((flags & GPUOS_START_DRAIN) ? KF_DRAIN : 0u) | ((rt->cfg.flags & GPUOS_CFG_TRACE) ? KF_TRACE : 0u) |
             ((rt->cfg.flags & GPUOS_CFG_NO_BULK) ? KF_NO_BULK : 0u);
   p.grid = rt->grid;
+  // Entries of this session not yet in the device ring: copied now (drained
+  // sessions) or fetched by the kernel (live sessions).
+  if (flags & GPUOS_START_DRAIN) {
+    const u64 from = std::max(rt->dma_upto, base);
+    if (from < rt->published && !dma_ring(rt, from, rt->published)) {
+      rt->sticky = GPUOS_EDEVICE;
+      return GPUOS_EDEVICE;
+    }
+  }
+  if (rt->dma_upto > base && cudaStreamWaitEvent(rt->stream, rt->dma_ev, 0) != cudaSuccess) {
+    rt->sticky = GPUOS_EDEVICE;
+    return GPUOS_EDEVICE;
+  }
+  p.fetched_upto = std::min(std::max(rt->dma_upto, base), rt->published);
   const int e = launch_session(p, rt->published, big_init, rt->stream);
   if (e != 0) {
     rt->sticky = GPUOS_EDEVICE;
@@ -279,7 +313,18 @@ gpuos_status start_kernel(gpuos* rt, u32 flags) {
 gpuos_status publish(gpuos* rt) {
   _mm_sfence();
   __atomic_store_n(&rt->hctl->head, rt->next_id, __ATOMIC_RELEASE);
+  const u64 old = rt->published;
   rt->published = rt->next_id;
+  // With no kernel running, or a drained one (which never reads ids at or
+  // past its own head), the new entries go to the device ring right away. A
+  // live kernel copies them itself.
+  if (!rt->running || (rt->run_flags & GPUOS_START_DRAIN)) {
+    const u64 from = std::max(rt->dma_upto, old);
+    if (from < rt->published && !dma_ring(rt, from, rt->published)) {
+      rt->sticky = GPUOS_EDEVICE;
+      return GPUOS_EDEVICE;
+    }
+  }
   return GPUOS_OK;
 }
 
@@ -429,6 +474,7 @@ void free_all(gpuos* rt) {
   if (rt->mctl) cudaFree(rt->mctl);
   if (rt->cstats) cudaFree(rt->cstats);
   if (rt->trace) cudaFree(rt->trace);
+  if (rt->dma_ev) cudaEventDestroy(rt->dma_ev);
   if (rt->aux) cudaStreamDestroy(rt->aux);
 }
 
@@ -473,6 +519,7 @@ gpuos_status gpuos_create_ex(gpuos_stream_t stream, const gpuos_config* cfg_in, 
   rt->cap = cfg.ring_capacity;
   rt->mask = rt->cap - 1;
   bool ok = cudaStreamCreateWithFlags(&rt->aux, cudaStreamNonBlocking) == cudaSuccess;
+  ok = ok && cudaEventCreateWithFlags(&rt->dma_ev, cudaEventDisableTiming) == cudaSuccess;
   ok = ok && cudaHostAlloc((void**)&rt->hring, rt->cap * sizeof(RingEntry),
                            cudaHostAllocMapped | cudaHostAllocWriteCombined) == cudaSuccess;
   ok = ok && cudaHostAlloc((void**)&rt->hctl, sizeof(HostCtl), cudaHostAllocMapped) == cudaSuccess;

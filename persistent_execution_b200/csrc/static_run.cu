@@ -163,6 +163,7 @@ extern "C" gpuos_status gpuos_run_static(const gpuos_desc* descs, uint64_t n, co
   p.mctl = nullptr;
   p.mask = STATIC_MAX_OPS - 1;
   p.base = 0;
+  p.fetched_upto = 0;  // the fetchers copy the entries onto themselves
   p.timeout_ns = cfg.timeout_ns;
   p.idle_exit_ns = cfg.idle_exit_ns;
   p.elem_chunk = cfg.elem_chunk;
