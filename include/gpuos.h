@@ -8,11 +8,11 @@
  * library is that primitive, re-designed for B200:
  *   - the host writes 128-byte op descriptors into a ring in mapped pinned
  *     memory and publishes a head counter (one doorbell per batch, in place of
- *     the per-launch doorbell of "Kernel Launch and Host-Device Interaction",
- *     section 5 "The launch path", steps 3-4);
+ *     the per-launch ring write and doorbell of "Kernel Launch and
+ *     Host-Device Interaction", section 5, "The launch path");
  *   - one persistent kernel, one CTA per SM, copies descriptors into device
- *     memory, claims ops and work items of large ops with atomics ("a
- *     persistent worker kernel with atomic task queues", GPUOS abstract),
+ *     memory, claims ops and work items of large ops with atomics (the
+ *     persistent worker and atomic task queues of the GPUOS abstract),
  *     waits for up to two dependencies per op through per-op completion words
  *     with acquire/release ordering, and runs each op body from an
  *     ahead-of-time opcode switch or a fused micro-op program held in

@@ -9,11 +9,12 @@
  *
  * Sources of each definition:
  *  - relu(a*x+b): "Launch Overhead and Fusion", section "Fusion" (the fused
- *    multiply, add, relu chain) and the fusion.go listing's constants.
+ *    multiply, add, relu chain) and the worked example of that page's demo.
  *  - add, mul, scale, gelu (erf form), silu*mul, row sum/max, softmax,
- *    RMSNorm, LayerNorm, rotary (half-split pairs, base 10000): the pages only
- *    name the op classes (GPUOS abstract: "small tensor operations ...
- *    attention patterns"); the formulas are the standard definitions.
+ *    RMSNorm, LayerNorm, rotary (half-split pairs, base 10000): the pages name
+ *    only the classes of ops (the GPUOS page, "The Paper": many small tensor
+ *    ops of inference and attention); the formulas are the standard
+ *    definitions.
  * Build: gcc -O2 -ffp-contract=off -fPIC -shared oracle.c -lm
  */
 #include "oracle.h"

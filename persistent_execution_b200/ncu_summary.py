@@ -67,14 +67,24 @@ def launches(path) -> str:
     return "\n".join(out)
 
 
+def _col(hdr, name):
+    """Column of a metric in a raw-page header, whose names may carry a section prefix."""
+    if name in hdr:
+        return hdr.index(name)
+    for i, h in enumerate(hdr):
+        if h.endswith("." + name):
+            return i
+    return -1
+
+
 def raw(path, names=DEFAULT_RAW) -> str:
     rows = list(csv.reader(open(path)))
     hdr, units = rows[0], rows[1]
     out = ["| metric | value | unit |", "|---|---:|---|"]
     for r in rows[2:]:
         for n in names:
-            if n in hdr:
-                i = hdr.index(n)
+            i = _col(hdr, n)
+            if i >= 0:
                 out.append(f"| `{n}` | {r[i]} | {units[i]} |")
     return "\n".join(out)
 
@@ -90,7 +100,7 @@ def dram_bytes(path) -> float:
     rows = list(csv.reader(open(path)))
     if rows and rows[0] and rows[0][0] == "ID" and "Metric Name" not in rows[0]:  # raw page
         hdr, units, vals = rows[0], rows[1], rows[2]
-        return sum(_to_bytes(vals[hdr.index(m)], units[hdr.index(m)])
+        return sum(_to_bytes(vals[_col(hdr, m)], units[_col(hdr, m)])
                    for m in ("dram__bytes_read.sum", "dram__bytes_write.sum"))
     hdr, data = _table(path)
     ki, mi, ui, vi = (hdr.index("Kernel Name"), hdr.index("Metric Name"), hdr.index("Metric Unit"),
