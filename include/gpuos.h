@@ -128,8 +128,8 @@ typedef struct gpuos_config {
   uint64_t timeout_ns;      /* budget of every device wait on another op. Default 2 s */
   uint64_t submit_timeout_ns; /* how long gpuos_submit waits for ring space. Default 2 s */
   uint64_t idle_exit_ns;    /* kernel exits after this long with nothing to do (flush relaunches it). Default 20 s */
-  uint32_t elem_chunk;      /* elements per work item of elementwise ops; multiple of 1024. Default 65536 */
-  uint32_t row_chunk;       /* target elements per work item of row ops; rows per item = clamp(row_chunk/cols, 1, 1024). Default 65536 */
+  uint32_t elem_chunk;      /* elements per work item of elementwise ops; multiple of 1024. Default 262144 */
+  uint32_t row_chunk;       /* target elements per work item of row ops; rows per item = clamp(row_chunk/cols, 1, 1024). Default 524288 */
   uint32_t backoff_ns;      /* longest sleep of an idle poll. Default 1000 */
   uint32_t flags;           /* GPUOS_CFG_* */
 } gpuos_config;

@@ -121,8 +121,8 @@ void default_config(gpuos_config* c) {
   c->timeout_ns = 2000000000ull;
   c->submit_timeout_ns = 2000000000ull;
   c->idle_exit_ns = 20000000000ull;
-  c->elem_chunk = 65536;
-  c->row_chunk = 65536;
+  c->elem_chunk = 262144;  // large ops: few, long items (fewer claims; the grid streams HBM)
+  c->row_chunk = 524288;
   c->backoff_ns = 1000;
   c->flags = 0;
 }

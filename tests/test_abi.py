@@ -90,13 +90,14 @@ def test_validate_accepts_and_rejects():
 
 def test_work_items():
     wi = G.gpuos_work_items
-    assert wi(desc(cols=65536)) == 1
-    assert wi(desc(cols=65537)) == 2
-    assert wi(desc(cols=64 << 20)) == 1024
-    assert wi(desc("rowsum", rows=8192, cols=8192)) == 1024   # 8 rows per item
+    assert wi(desc(cols=262144)) == 1
+    assert wi(desc(cols=262145)) == 2
+    assert wi(desc(cols=64 << 20)) == 256
+    assert wi(desc("rowsum", rows=8192, cols=8192)) == 128    # 64 rows per item
     assert wi(desc("softmax", rows=8, cols=4096)) == 1
     assert wi(desc("layernorm", rows=3000, cols=64)) == 3       # at most 1024 rows per item
-    assert wi(desc("rowmax", rows=5, cols=200000)) == 5         # one row per item at least
+    assert wi(desc("rowmax", rows=5, cols=200000)) == 3         # two rows per item
+    assert wi(desc("rowmax", rows=5, cols=600000)) == 5         # one row per item at least
     cfg = G.default_config(elem_chunk=4096)
     assert wi(desc(cols=4097), cfg) == 2
     assert wi(desc(opcode=99)) == 0

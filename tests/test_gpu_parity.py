@@ -29,7 +29,7 @@ def need_gpu():
 
 
 # ------------------------------------------------------------------ single ops, edge sizes
-EW_SIZES = [1, 3, 8, 4095, 4097, 65536, 3 * 65536 + 37]
+EW_SIZES = [1, 3, 8, 4095, 4097, 65536, 3 * 65536 + 37, 3 * 262144 + 37]
 EW_CASES = [("add", {}), ("mul", {}), ("scale", dict(scalars=(-1.75, 0, 0, 0))),
             ("gelu", {}), ("relu_affine", dict(scalars=(1.3, -0.2, 0, 0))), ("silu_mul", {}),
             ("ew_chain", dict(scalars=(0.7, 0.1, 2.0, 0), prog=("affine", "relu", "add1", "scale", "mul2"))),
@@ -56,7 +56,8 @@ def test_elementwise_edge_sizes(kind, kw, dtype):
 
 @pytest.mark.parametrize("dtype", [0, 1])
 def test_elementwise_broadcast(dtype):
-    for n, n0, n1 in [(1000, 7, 1000), (4097, 4097, 13), (65536 * 2 + 5, 65536 * 2 + 5, 3000), (96, 8, 16)]:
+    for n, n0, n1 in [(1000, 7, 1000), (4097, 4097, 13), (65536 * 2 + 5, 65536 * 2 + 5, 3000), (96, 8, 16),
+                      (600000, 600000, 3000)]:
         for kind in ("add", "mul", "silu_mul"):
             w = W.single_op(kind, dtype, 1, n, bcast=(n0, n1), seed=n + n1)
             _, _, _, _, f, fb = _run_both(w)
