@@ -92,6 +92,7 @@ struct Control {
   u64 claimed = 0, runops = 0, idle_cyc = 0, dep_cyc = 0, fetched = 0;
   u64 mb_head = 0;                // mailbox slots this CTA has taken
   u64 held = 0;                   // id + 1 of the single op claimed here and not yet emitted
+  bool contended = false;         // this CTA lost a CAS claim race in this session (lane 0)
   u32 ndef = 0;                   // entries of S->deferred
   const bool drain;
 
@@ -663,16 +664,24 @@ struct Control {
     u64 c2 = 0;
     uint4 chunk = uint4{0, 0, 0, 0};
     if (lane == 0) {
-      if (hm - c > 2ull * p.grid + 64ull) {
+      // Near the head, claims take the peeked id by CAS: none runs ahead of
+      // what the host published, and a FOLLOW op is left to its predecessor's
+      // CTA. A drained session's head is fixed, so once this CTA has lost a
+      // CAS race it claims by atomicAdd there too (a claim past the head is
+      // simply empty); CAS contention would otherwise serialise the last
+      // few hundred claims.
+      if ((drain && contended && !hdr_follow(h)) || hm - c > 2ull * p.grid + 64ull) {
         c2 = atomicAdd(&p.st->next_op.v, 1ull);
       } else {
         c2 = atomicCAS(&p.st->next_op.v, c, c + 1) == c ? c : ~0ull;
+        if (c2 == ~0ull) contended = true;
       }
     }
     if (lane < 8) chunk = __ldcg(reinterpret_cast<const uint4*>(ent(c)) + lane);
     if (lane == 0 && c2 != ~0ull) st_relaxed_gpu(&p.st->activity.v, globaltimer());
     c2 = bcast(c2);
     if (c2 == ~0ull) return 2;
+    if (drain && c2 >= hm) return 0;
     ++claimed;
     backoff = 0;
     if (c2 != c) {
