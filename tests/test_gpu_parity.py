@@ -134,6 +134,40 @@ def test_chain_affinity_keeps_chains_on_one_cta():
     assert len(np.unique(tr["cta"])) <= 3
 
 
+@pytest.mark.parametrize("dtype", [0, 1])
+@pytest.mark.parametrize("n", [4096, 2048, 8192, 256 * 16 * 12, 4100, 300])
+def test_dependent_elementwise_chains_bit_exact(dtype, n):
+    # Chains of fused relu-affine ops and adds, each reading the previous
+    # output as its first or second operand, at sizes of whole tiles, partial
+    # warps and ragged tails. Every output must equal the oracle's, bit for bit.
+    b = W._Builder("forwarding", 5)
+    rng = b.rng
+
+    def data():
+        v = rng.standard_normal(n, dtype=np.float32)
+        return v if dtype == 0 else W.bf16_bits_trunc(v)
+
+    src = b.alloc_input(dtype, data())
+    other = b.alloc_input(dtype, data())
+    prev = -1
+    for i in range(60):
+        out = b.alloc_output(dtype, n)
+        if i % 5 == 4:  # the previous output as second operand
+            prev = b.add_op("add", dtype, [other, src], out, 1, n, in_n=(n, n), deps=[prev])
+        elif i % 3 == 2:
+            prev = b.add_op("add", dtype, [src, other], out, 1, n, in_n=(n, n), deps=[prev])
+        else:
+            a, c = rng.uniform(-1.5, 1.5, 2)
+            prev = b.add_op("ew_chain", dtype, [src], out, 1, n, in_n=(n, 0), s=(a, c, 0, 0),
+                            prog=("affine", "relu"), deps=[prev])
+        src = out
+    w = b.finish({})
+    a32, a16, _, _ = U.run_persistent(w)
+    assert not P.check_ops(w, a32, a16)
+    r32, r16 = oracle.run(w)
+    assert P.bit_exact(w, a32, a16, r32, r16) == []
+
+
 @pytest.mark.parametrize("mode", ["drain", "live"])
 def test_chain_handoff_interleaved_streams(mode):
     # config 4's request chains are interleaved, so a claimed op's predecessor
