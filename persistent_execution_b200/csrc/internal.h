@@ -103,12 +103,14 @@ struct DevState {
   Line activity;     // globaltimer of the last claim
   Line span_start;   // min item start
   Line span_end;     // max item end
+  Line dma_mirror;   // dma_head as last read by the device
 };
 
 // Host control block in mapped pinned memory.
 struct HostCtl {
   volatile u64 head;  // host -> device: ops [0, head) are published
-  u64 pad0[15];
+  volatile u64 dma_head;  // host -> device: entries [0, dma_head) were copied into the device ring by the host
+  u64 pad0[14];
   volatile u64 stop;        // host -> device
   volatile u64 stall_gate;  // host -> device: nonzero lets STALL ops finish
   u64 pad1[14];

@@ -385,9 +385,16 @@ struct Control {
         got = fn < hm;
         if (!got) e = fn;
       } else if (fn < hm) {
-        e = fn + 32 < hm ? fn + 32 : hm;
-        got = atomicCAS(&p.st->fetch_next.v, fn, e) == fn;
-        if (!got) e = fn + 1;  // someone else took it: still progress
+        const u64 dm = ld_acquire_gpu(&p.st->dma_mirror.v);
+        if (fn < dm) {
+          // the host already copied these entries into the device ring: skip them
+          atomicCAS(&p.st->fetch_next.v, fn, dm);
+          e = fn + 1;  // progress, nothing to copy
+        } else {
+          e = fn + 32 < hm ? fn + 32 : hm;
+          got = atomicCAS(&p.st->fetch_next.v, fn, e) == fn;
+          if (!got) e = fn + 1;  // someone else took it: still progress
+        }
       }
     }
     fn = bcast(fn);
@@ -425,7 +432,9 @@ struct Control {
     if (now - ld_relaxed_gpu(&p.st->poll_time.v) < 1000) return;
     if (atomicCAS(&p.st->poll_lock.v, 0ull, 1ull) != 0) return;
     const u64 h = ld_acquire_sys(&p.hctl->head);
+    const u64 dh = ld_relaxed_sys(&p.hctl->dma_head);  // written before head
     const u64 sp = ld_relaxed_sys(&p.hctl->stop);
+    if (dh > ld_relaxed_gpu(&p.st->dma_mirror.v)) atom_max_release_gpu(&p.st->dma_mirror.v, dh);
     if (h > ld_relaxed_gpu(&p.st->head_mirror.v)) atom_max_release_gpu(&p.st->head_mirror.v, h);
     if (sp) st_release_gpu(&p.st->stop.v, 1ull);
     st_relaxed_gpu(&p.st->poll_time.v, globaltimer());
@@ -950,6 +959,7 @@ __global__ void gpuos_reset_kernel(const KParams p, u64 head, u64 big_init) {
     DevState* st = p.st;
     st->next_op.v = p.base;
     st->fetch_next.v = p.fetched_upto > p.base ? p.fetched_upto : p.base;
+    st->dma_mirror.v = st->fetch_next.v;
     st->head_mirror.v = head;
     st->big.v = big_init;
     st->poll_lock.v = 0;

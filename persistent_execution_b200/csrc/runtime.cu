@@ -310,14 +310,30 @@ gpuos_status start_kernel(gpuos* rt, u32 flags) {
   return GPUOS_OK;
 }
 
+// Flushes of at least this many new ops to a live kernel are copied into the
+// device ring by the copy engine before the head moves; smaller ones are
+// fetched by the kernel's control warps.
+constexpr u64 LIVE_DMA_MIN = 128;
+
 gpuos_status publish(gpuos* rt) {
   _mm_sfence();
-  __atomic_store_n(&rt->hctl->head, rt->next_id, __ATOMIC_RELEASE);
   const u64 old = rt->published;
+  const bool live = rt->running && !(rt->run_flags & GPUOS_START_DRAIN);
+  if (live && rt->next_id - old >= LIVE_DMA_MIN) {
+    // Every entry of the session not yet copied goes now (entries the kernel
+    // fetched itself are rewritten with the same bytes); the head moves only
+    // after the copy completed, so the kernel never reads a partial entry.
+    const u64 from = std::max(rt->dma_upto, rt->session_base);
+    if (!dma_ring(rt, from, rt->next_id) || cudaEventSynchronize(rt->dma_ev) != cudaSuccess) {
+      rt->sticky = GPUOS_EDEVICE;
+      return GPUOS_EDEVICE;
+    }
+    __atomic_store_n(&rt->hctl->dma_head, rt->next_id, __ATOMIC_RELEASE);
+  }
+  __atomic_store_n(&rt->hctl->head, rt->next_id, __ATOMIC_RELEASE);
   rt->published = rt->next_id;
   // With no kernel running, or a drained one (which never reads ids at or
-  // past its own head), the new entries go to the device ring right away. A
-  // live kernel copies them itself.
+  // past its own head), the new entries go to the device ring right away.
   if (!rt->running || (rt->run_flags & GPUOS_START_DRAIN)) {
     const u64 from = std::max(rt->dma_upto, old);
     if (from < rt->published && !dma_ring(rt, from, rt->published)) {
