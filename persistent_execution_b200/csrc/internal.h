@@ -62,7 +62,8 @@ GPUOS_HD bool op_is_ew(int op) {
 }
 
 GPUOS_HD long long rows_per_item(long long cols, u32 row_chunk) {
-  long long r = (long long)row_chunk / cols;
+  // 32-bit division when cols fits (it always does below 2^32 columns)
+  long long r = cols <= 0xffffffffll ? (long long)(row_chunk / (u32)cols) : 0;
   if (r < 1) r = 1;
   if (r > 1024) r = 1024;
   return r;

@@ -430,7 +430,8 @@ static __device__ __noinline__ void ew_loop(const RingEntry& E, u32 item, u32 el
     // t is now the first tile >= full that this warp owns: the partial last
     // tile, if any, takes the scalar layout below
   }
-  const long long s0 = n0 < n ? 32 % n0 : 32, s1 = (u1 && n1 < n) ? 32 % n1 : 32;
+  const long long s0 = n0 < n ? (long long)umod(32, (u64)n0) : 32;
+  const long long s1 = (u1 && n1 < n) ? (long long)umod(32, (u64)n1) : 32;
   for (; t < tiles; t += NW) {
     const long long t0 = e0 + t * EW_TILE;
     float a[8], b[8], c[8];
@@ -466,7 +467,7 @@ static __device__ __noinline__ void ew_stream(const RingEntry& E, u32 item, u32 
   const long long e1 = min(n, e0 + (long long)elem_chunk);
   const long long nchunks = (e1 - e0 + CE - 1) / CE;
   const int w = cx.warp, NW = cx.nwarps, lane = cx.lane;
-  const int mine = nchunks > w ? (int)((nchunks - w + NW - 1) / NW) : 0;
+  const int mine = nchunks > w ? (int)((u32)(nchunks - w + NW - 1) / (u32)NW) : 0;  // nchunks <= elem_chunk / 256
   if (mine == 0) return;
   const unsigned base = cx.ws->seq;
   __syncwarp();
@@ -872,8 +873,8 @@ static __device__ __noinline__ void row_staged(const RingEntry& E, u32 item, u32
   const int R = (int)min(rpi, rows - r0);
   constexpr int op = OP;
   int S = 1;
-  while (2 * S * R <= cx.nwarps && cols / (2 * S) >= 256) S *= 2;
-  long long seg = (cols + S - 1) / S;
+  while (2 * S * R <= cx.nwarps && cols >= 512ll * S) S *= 2;  // cols / (2S) >= 256, without a division
+  long long seg = (cols + S - 1) >> (__ffs(S) - 1);                 // S is a power of two
   seg = (seg + 7) & ~7ll;
   const int tasks = R * S;
   const int nwv = op == GPUOS_OP_RMSNORM ? 1 : (op == GPUOS_OP_LAYERNORM ? 2 : 0);
@@ -1069,8 +1070,10 @@ static __device__ __noinline__ void rotary_item(const RingEntry& E, long long r0
   const double base = (double)E.s[0];
   long long ti = -1;  // the column pair whose angle is in cs, sn
   double cs = 0.0, sn = 0.0;
+  const bool narrow = total <= 0x7fffffffll;  // 32-bit index arithmetic
   for (long long p = cx.tid; p < total; p += cx.nthr) {
-    const long long row = p / half, i = p % half;
+    const long long row = narrow ? (long long)((u32)p / (u32)half) : p / half;
+    const long long i = narrow ? (long long)((u32)p % (u32)half) : p % half;
     if (i != ti) {  // the angle depends on the column pair only
       const double2 t = rotary_cs(base, i, cols, E.pos);
       cs = t.x;
@@ -1096,8 +1099,8 @@ static __device__ __noinline__ void row_item(const RingEntry& E, u32 item, u32 r
     return;
   }
   int S = 1;  // warps per row
-  while (2 * S * R <= cx.nwarps && cols / (2 * S) >= 256) S *= 2;
-  long long seg = (cols + S - 1) / S;
+  while (2 * S * R <= cx.nwarps && cols >= 512ll * S) S *= 2;  // cols / (2S) >= 256, without a division
+  long long seg = (cols + S - 1) >> (__ffs(S) - 1);                 // S is a power of two
   seg = (seg + 7) & ~7ll;
   const int tasks = R * S;
   bool vec = al16(E.in0) && (cols % 8) == 0;
