@@ -41,6 +41,7 @@ __global__ void __launch_bounds__(NCW * 32) gpuos_op_kernel(const RingEntry e, u
   cx.hctl = nullptr;
   cx.id = 0;
   cx.flags = 0;
+  cx.rot = nullptr;
   const OpEnv env{nullptr, nullptr, 0ull, 0ull};
   for (u64 it = blockIdx.x; it < n; it += gridDim.x) {
     run_item(E, (u32)it, elem_chunk, row_chunk, cx, env);

@@ -28,6 +28,18 @@ struct __align__(128) WarpSmem {
   unsigned seq;  // stage uses so far, modulo 6: use u lives in stage u % 3 with phase parity (u / 3) & 1
 };
 
+// Rotation angles of the last rotary op this CTA ran: cos and sin of
+// pos * base^(-2i/cols) for each column pair i. Consecutive rotary ops with the
+// same base, width and position (q and k of every layer of a decode step) reuse
+// them instead of recomputing them in double precision.
+constexpr int ROT_MAX_PAIRS = 256;
+struct RotCache {
+  float base;
+  int pos;
+  long long cols;  // 0: empty
+  double2 cs[ROT_MAX_PAIRS];
+};
+
 struct Cx {
   int tid, nthr;       // thread index in the compute group, group size
   int warp, nwarps, lane;
@@ -38,6 +50,7 @@ struct Cx {
   HostCtl* hctl;
   u64 id;              // op id, for error reports
   u32 flags;           // KF_* of the launch (KF_NO_BULK: register paths only)
+  RotCache* rot;       // shared rotary angle cache, or null
 };
 
 struct OpEnv {
@@ -874,7 +887,8 @@ static __device__ __noinline__ void row_staged(const RingEntry& E, u32 item, u32
   constexpr int op = OP;
   int S = 1;
   while (2 * S * R <= cx.nwarps && cols >= 512ll * S) S *= 2;  // cols / (2S) >= 256, without a division
-  long long seg = (cols + S - 1) >> (__ffs(S) - 1);                 // S is a power of two
+  const int lgS = __ffs(S) - 1;                                     // S is a power of two
+  long long seg = (cols + S - 1) >> lgS;
   seg = (seg + 7) & ~7ll;
   const int tasks = R * S;
   const int nwv = op == GPUOS_OP_RMSNORM ? 1 : (op == GPUOS_OP_LAYERNORM ? 2 : 0);
@@ -894,7 +908,7 @@ static __device__ __noinline__ void row_staged(const RingEntry& E, u32 item, u32
     // one stage use per task; mode 0 keeps three tasks in flight
     auto issue = [&](int i) {  // lane 0
       const int t = w + i * NW;
-      const int row = t / S, sg = t % S;
+      const int row = t >> lgS, sg = t & (S - 1);
       const long long c0 = (long long)sg * seg, c1 = min(cols, c0 + seg);
       const unsigned xb = (unsigned)((c1 - c0) * ES);
       const unsigned uu = base + (unsigned)i;
@@ -912,7 +926,7 @@ static __device__ __noinline__ void row_staged(const RingEntry& E, u32 item, u32
     }
     for (int i = 0; i < mine; ++i) {
       const int t = w + i * NW;
-      const int row = t / S, sg = t % S;
+      const int row = t >> lgS, sg = t & (S - 1);
       const long long c0 = (long long)sg * seg, c1 = min(cols, c0 + seg);
       const int ne = (int)(c1 - c0);
       const unsigned uu = base + (unsigned)i;
@@ -942,7 +956,7 @@ static __device__ __noinline__ void row_staged(const RingEntry& E, u32 item, u32
       cx_sync(cx);
       if (mine == 1) {
         const int t = w;
-        const int row = t / S, sg = t % S;
+        const int row = t >> lgS, sg = t & (S - 1);
         const long long c0 = (long long)sg * seg, c1 = min(cols, c0 + seg);
         const int ne = (int)(c1 - c0);
         const float4 q0 = cx.part[row * S];
@@ -1008,7 +1022,7 @@ static __device__ __noinline__ void row_staged(const RingEntry& E, u32 item, u32
     };
     for (int i = 0; i < mine; ++i) {
       const int t = w + i * NW;
-      const int row = t / S, sg = t % S;
+      const int row = t >> lgS, sg = t & (S - 1);
       const long long c0 = (long long)sg * seg, c1 = min(cols, c0 + seg);
       const long long gs = (r0 + row) * cols + c0;
       const float K = op == GPUOS_OP_LAYERNORM ? ld1<DT>(E.in0, (r0 + row) * cols) : 0.f;
@@ -1031,7 +1045,7 @@ static __device__ __noinline__ void row_staged(const RingEntry& E, u32 item, u32
       cx_sync(cx);
       if (mine == 1) {
         const int t = w;
-        const int row = t / S, sg = t % S;
+        const int row = t >> lgS, sg = t & (S - 1);
         const long long c0 = (long long)sg * seg, c1 = min(cols, c0 + seg);
         const float4 q0 = cx.part[row * S];
         Acc A{q0.x, q0.y};
@@ -1071,11 +1085,24 @@ static __device__ __noinline__ void rotary_item(const RingEntry& E, long long r0
   long long ti = -1;  // the column pair whose angle is in cs, sn
   double cs = 0.0, sn = 0.0;
   const bool narrow = total <= 0x7fffffffll;  // 32-bit index arithmetic
+  RotCache* rc = (cx.rot != nullptr && half <= ROT_MAX_PAIRS) ? cx.rot : nullptr;
+  if (rc) {
+    const bool hit = rc->cols == cols && rc->pos == E.pos && rc->base == E.s[0];
+    if (!hit) {
+      for (long long i = cx.tid; i < half; i += cx.nthr) rc->cs[i] = rotary_cs(base, i, cols, E.pos);
+      cx_sync(cx);
+      if (cx.tid == 0) {  // read by the next rotary op, after this item's closing barrier
+        rc->cols = cols;
+        rc->pos = E.pos;
+        rc->base = E.s[0];
+      }
+    }
+  }
   for (long long p = cx.tid; p < total; p += cx.nthr) {
     const long long row = narrow ? (long long)((u32)p / (u32)half) : p / half;
     const long long i = narrow ? (long long)((u32)p % (u32)half) : p % half;
     if (i != ti) {  // the angle depends on the column pair only
-      const double2 t = rotary_cs(base, i, cols, E.pos);
+      const double2 t = rc ? rc->cs[i] : rotary_cs(base, i, cols, E.pos);
       cs = t.x;
       sn = t.y;
       ti = i;
@@ -1100,7 +1127,8 @@ static __device__ __noinline__ void row_item(const RingEntry& E, u32 item, u32 r
   }
   int S = 1;  // warps per row
   while (2 * S * R <= cx.nwarps && cols >= 512ll * S) S *= 2;  // cols / (2S) >= 256, without a division
-  long long seg = (cols + S - 1) >> (__ffs(S) - 1);                 // S is a power of two
+  const int lgS = __ffs(S) - 1;                                     // S is a power of two
+  long long seg = (cols + S - 1) >> lgS;
   seg = (seg + 7) & ~7ll;
   const int tasks = R * S;
   bool vec = al16(E.in0) && (cols % 8) == 0;
@@ -1110,7 +1138,7 @@ static __device__ __noinline__ void row_item(const RingEntry& E, u32 item, u32 r
   const bool stats_only = (op == GPUOS_OP_ROWSUM || op == GPUOS_OP_ROWMAX);
 
   for (int t = cx.warp; t < tasks; t += cx.nwarps) {
-    const int row = t / S, sg = t % S;
+    const int row = t >> lgS, sg = t & (S - 1);
     const long long c0 = (long long)sg * seg, c1 = min(cols, c0 + seg);
     const long long rb = (r0 + row) * cols;
     const float K = (op == GPUOS_OP_LAYERNORM) ? ld1<DT>(E.in0, rb) : 0.f;
@@ -1139,7 +1167,7 @@ static __device__ __noinline__ void row_item(const RingEntry& E, u32 item, u32 r
   if (S > 1) {
     cx_sync(cx);
     for (int t = cx.warp; t < tasks; t += cx.nwarps) {
-      const int row = t / S, sg = t % S;
+      const int row = t >> lgS, sg = t & (S - 1);
       const long long c0 = (long long)sg * seg, c1 = min(cols, c0 + seg);
       const long long rb = (r0 + row) * cols;
       const float4 q0 = cx.part[row * S];

@@ -66,6 +66,7 @@ struct Smem {
   float4 part[NCW];
   u64 recent[8];
   u64 deferred[32];         // mailbox ops waiting for the op this CTA holds (ids)
+  RotCache rot;             // rotary angles of the last rotary op
   volatile unsigned ncomp;  // items the compute warps finished
 };
 constexpr u32 DEFER = 32;
@@ -893,6 +894,7 @@ __device__ void compute(const KParams& p, Smem* S, WarpSmem* W, int warp, int la
   cx.hctl = p.hctl;
   cx.id = 0;
   cx.flags = p.flags;
+  cx.rot = &S->rot;
   const bool leader = cx.tid == 0;
   for (u64 k = 0;; ++k) {
     const u32 slot = (u32)(k % FIFO);
@@ -930,6 +932,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gpuos_persistent_kernel(const __g
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     S.ncomp = 0;
+    S.rot.cols = 0;
     for (int i = 0; i < FIFO; ++i) {
       mbar_init(&S.full_bar[i], 1);
       mbar_init(&S.done_bar[i], 1);
