@@ -592,7 +592,7 @@ __device__ void ew_item(const RingEntry& E, u32 item, u32 elem_chunk, const Cx& 
     case GPUOS_OP_SCALE: ew_loop<DT, GPUOS_OP_SCALE, 2 * EW_UNR, 0>(E, item, elem_chunk, cx); break;
     case GPUOS_OP_GELU: ew_loop<DT, GPUOS_OP_GELU, 1, 0>(E, item, elem_chunk, cx); break;
     case GPUOS_OP_RELU_AFFINE: ew_loop<DT, GPUOS_OP_RELU_AFFINE, 2 * EW_UNR, 0>(E, item, elem_chunk, cx); break;
-    case GPUOS_OP_SILU_MUL: ew_loop<DT, GPUOS_OP_SILU_MUL, 1, 1>(E, item, elem_chunk, cx); break;
+    case GPUOS_OP_SILU_MUL: ew_loop<DT, GPUOS_OP_SILU_MUL, EW_UNR, 1>(E, item, elem_chunk, cx); break;
     default:
       if (chain_calls(E)) {
         ew_loop<DT, OPK_CHAIN_CALLS, 1, -1>(E, item, elem_chunk, cx);
