@@ -260,13 +260,18 @@ struct Control {
   // to the CTA that emitted its one unfinished dependency. True if posted;
   // false leaves c to the caller (nothing to wait for, two unfinished
   // dependencies, an unknown or local owner, or a full mailbox).
-  __device__ __forceinline__ bool try_handoff(u64 c, u64 d0, u64 d1) {
-    if (!p.mbox || (d0 | d1) == 0) return false;
-    if ((d0 != 0 && is_local(d0 - 1)) || (d1 != 0 && is_local(d1 - 1))) return false;
-    u32 ok = 0;
+  // HO_POSTED: posted. HO_READY: every dependency already completed (read with
+  // acquire ordering, so the caller needs no wait). HO_NONE: the caller waits.
+  enum { HO_NONE = 0, HO_POSTED = 1, HO_READY = 2 };
+  __device__ __forceinline__ int try_handoff(u64 c, u64 d0, u64 d1) {
+    if ((d0 | d1) == 0) return HO_READY;
+    if (!p.mbox) return HO_NONE;
+    if ((d0 != 0 && is_local(d0 - 1)) || (d1 != 0 && is_local(d1 - 1))) return HO_NONE;
+    u32 ok = HO_NONE;
     if (lane == 0) {
       const bool u0 = d0 != 0 && ld_acquire_gpu(&p.done[(d0 - 1) & p.mask]) < d0;
       const bool u1 = d1 != 0 && ld_acquire_gpu(&p.done[(d1 - 1) & p.mask]) < d1;
+      if (!u0 && !u1) ok = HO_READY;
       if (u0 != u1) {
         const u64 a = u0 ? d0 : d1;
         const u64 o = ld_relaxed_gpu(&p.owner[(a - 1) & p.mask]);
@@ -279,12 +284,12 @@ struct Control {
             st_release_gpu(&p.mbox[(u64)cta * MAILBOX + (t % MAILBOX)], c + 1);
             // c is owned there from now on: its own dependants follow it
             st_relaxed_gpu(&p.owner[c & p.mask], ((c + 1) << 16) | (u64)cta);
-            ok = 1;
+            ok = HO_POSTED;
           }
         }
       }
     }
-    return bcast32(ok) != 0;
+    return (int)bcast32(ok);
   }
 
   // Waits until this CTA has fewer than `lim` items emitted but not finished.
@@ -538,12 +543,14 @@ struct Control {
     }
     d0 = bcast(d0);
     d1 = bcast(d1);
+    int ho = HO_NONE;
     if (handoff) {
-      if (try_handoff(c, d0, d1)) return 2;
+      ho = try_handoff(c, d0, d1);
+      if (ho == HO_POSTED) return 2;
       held = c + 1;  // dependants may be posted here from now on
       set_owner(c);
     }
-    if (!wait_deps(c, d0, d1)) return 0;
+    if (ho != HO_READY && !wait_deps(c, d0, d1)) return 0;
     if (!emit(c, 0, 1, claim, staged)) return 0;
     note_single(c);
     set_owner(c);
@@ -694,6 +701,21 @@ struct Control {
     if (drain && c2 >= hm) return 0;
     ++claimed;
     backoff = 0;
+    if (c2 != c && drain) {
+      // A drained session's entries were all in the device ring before launch:
+      // the tag, the dependencies and the entry come in one round trip.
+      if (lane < 8) chunk = __ldcg(reinterpret_cast<const uint4*>(ent(c2)) + lane);
+      const u64 h2 = __shfl_sync(FULLMASK, (u64)chunk.x | ((u64)chunk.y << 32), 0);
+      if (hdr_tag(h2) == c2 + 1) {
+        if (hdr_items(h2) > 1) {
+          pending = c2 + 1;
+          pend_word = ~0ull;
+          return 1;
+        }
+        c = c2;  // continue below as if c2 had been the peeked op
+        h = h2;
+      }
+    }
     if (c2 != c) {
       if (!wait_fetched(c2, h)) return -1;
       if (hdr_items(h) > 1) {
@@ -714,10 +736,11 @@ struct Control {
     // dependencies straight from the entry in registers (dep0: lane 0, dep1: lane 1)
     const u64 d0 = __shfl_sync(FULLMASK, (u64)chunk.z | ((u64)chunk.w << 32), 0);
     const u64 d1 = __shfl_sync(FULLMASK, (u64)chunk.x | ((u64)chunk.y << 32), 1);
-    if (try_handoff(c, d0, d1)) return 1;
+    const int ho = try_handoff(c, d0, d1);
+    if (ho == HO_POSTED) return 1;
     held = c + 1;  // dependants may be posted here from now on
     set_owner(c);
-    if (!wait_deps(c, d0, d1)) return -1;
+    if (ho != HO_READY && !wait_deps(c, d0, d1)) return -1;
     if (!emit(c, 0, 1, CLAIM_SHARED, nullptr, true, chunk)) return -1;
     note_single(c);
     if (!release_held()) return -1;
