@@ -41,8 +41,10 @@ constexpr int FIFO = 8;
 // Items a CTA may have emitted but not finished before it claims another op
 // or joins a large op: a shallow window keeps ready ops from queueing behind
 // unrelated ones and keeps a large op's items from being hoarded long before
-// they run. Runs of FOLLOW ops use the whole FIFO.
-constexpr unsigned LOOKAHEAD = 2;
+// they run, while a claim (several round trips) still overlaps the items
+// ahead of it. Runs of FOLLOW ops use the whole FIFO. (2 -> 4: the 20,000-op
+// DAG 1.13 -> 1.03 ms; chains and the serving stream unchanged.)
+constexpr unsigned LOOKAHEAD = 4;
 constexpr unsigned FULLMASK = 0xffffffffu;
 
 enum : u32 { SLOT_WORK = 0, SLOT_EXIT = 1 };
