@@ -45,6 +45,7 @@ constexpr int FIFO = 8;
 // ahead of it. Runs of FOLLOW ops use the whole FIFO. (2 -> 4: the 20,000-op
 // DAG 1.13 -> 1.03 ms; chains and the serving stream unchanged.)
 constexpr unsigned LOOKAHEAD = 4;
+constexpr unsigned LOOKAHEAD_BIG = 2;  // joining a large op (large-op stress: 16.5 ms at 4, 15.5 at 2)
 constexpr unsigned FULLMASK = 0xffffffffu;
 
 enum : u32 { SLOT_WORK = 0, SLOT_EXIT = 1 };
@@ -570,6 +571,9 @@ struct Control {
       if (cur != 0) {
         const u64 h = hdr_of(cur - 1);
         if (hdr_tag(h) == cur && cnt < hdr_items(h)) {
+          // a large op's items are taken with a shorter look-ahead than single
+          // ops, so that no CTA holds items of it long before they run
+          while ((unsigned)k - S->ncomp >= LOOKAHEAD_BIG) __nanosleep(20);
           const u64 v = atomicAdd(&p.st->big.v, 1ull);
           const u64 op1 = v >> 24, k2 = v & BIG_COUNT_MASK;
           const u64 h2 = (op1 == cur) ? h : (op1 ? hdr_of(op1 - 1) : 0ull);
