@@ -10,8 +10,10 @@
  *     memory and publishes a head counter (one doorbell per batch, in place of
  *     the per-launch ring write and doorbell of "Kernel Launch and
  *     Host-Device Interaction", section 5, "The launch path");
- *   - one persistent kernel, one CTA per SM, copies descriptors into device
- *     memory, claims ops and work items of large ops with atomics (the
+ *   - the descriptors reach a device ring by the copy engine (or, for small
+ *     flushes to a running kernel, by the kernel itself);
+ *   - one persistent kernel, one CTA per SM, claims ops and work items of
+ *     large ops with atomics (the
  *     persistent worker and atomic task queues of the GPUOS abstract),
  *     waits for up to two dependencies per op through per-op completion words
  *     with acquire/release ordering, and runs each op body from an
@@ -149,7 +151,7 @@ typedef struct gpuos_stats {
   uint64_t run_ops;           /* ops taken by chain affinity (claimed as a run by the CTA that ran the predecessor) */
   uint64_t idle_poll_cycles;  /* SM cycles spent polling with nothing to do, summed over CTAs */
   uint64_t dep_wait_cycles;   /* SM cycles spent waiting for another CTA's op, summed over CTAs */
-  uint64_t fetch_descs;       /* descriptors copied from the host ring */
+  uint64_t fetch_descs;       /* descriptors the kernel copied from the host ring itself */
   uint64_t max_ring_occupancy;
   uint64_t gpu_span_ns;       /* last session: first item start to last item end (device globaltimer) */
   uint64_t kernel_launches;   /* kernels launched by this runtime */
@@ -182,7 +184,9 @@ gpuos_status gpuos_create_ex(gpuos_stream_t stream, const gpuos_config* cfg, gpu
 /* Launches the persistent kernel again after gpuos_stop (or after create with
  * GPUOS_CFG_NO_AUTOSTART). With GPUOS_START_DRAIN it runs the ops published by
  * gpuos_flush before this call and exits by itself; ops submitted later wait
- * for the next start. Returns GPUOS_EINVAL if it is already running. */
+ * for the next start. Before a drained launch the session's descriptors are
+ * copied into device memory (ordered before the kernel on `stream`). Returns
+ * GPUOS_EINVAL if it is already running. */
 gpuos_status gpuos_start(gpuos_t* rt, uint32_t flags);
 
 /* Waits (up to timeout_ns) for the session's work -- every submitted op, or
@@ -215,7 +219,11 @@ gpuos_status gpuos_submit_n(gpuos_t* rt, const gpuos_desc* descs, uint64_t n, ui
 
 /* Publishes every submitted op to the device: one release fence and one store
  * of the head counter into mapped memory. Relaunches a kernel that left after
- * idling. */
+ * idling. The new descriptors reach device memory by the copy engine (on an
+ * internal stream) when no kernel or a drained one is running, and, for a live
+ * kernel, when at least 128 ops are new: this call then waits for that copy
+ * before moving the head, so the kernel never reads descriptors over PCIe
+ * while ops run. Smaller flushes to a live kernel are fetched by the kernel. */
 gpuos_status gpuos_flush(gpuos_t* rt);
 
 /* Waits until op `id` (GPUOS_ALL: every submitted op) and every earlier op
