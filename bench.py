@@ -328,6 +328,27 @@ def bench_gpu(args, rank, world, local):
         e2e = {"value": R.job_throughput(n, ranks, e2e_ms / 1e3), "unit": "ops/s", "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms}
 
+    # Through the live API: a resident kernel (gpuos_create), the whole stream
+    # submitted and flushed, wall time from the first submit to gpuos_wait(ALL).
+    live = None
+    try:
+        rt3 = G.Runtime(stream.cuda_stream, ring_capacity=cap, timeout_ns=10_000_000_000,
+                        idle_exit_ns=30_000_000_000)
+        tl = []
+        for rep in range(4):
+            t0 = time.perf_counter()
+            rt3.submit_n(descs, dep_base=0)
+            rt3.flush()
+            G.check(rt3.wait(G.ALL, 120.0), "live wait")
+            if rep > 0:
+                tl.append(time.perf_counter() - t0)
+        rt3.destroy()
+        stream.synchronize()
+        live = {"us_per_op": float(np.median(tl)) / n * 1e6, "ms_per_stream": float(np.median(tl)) * 1e3,
+                "what": "kernel resident (gpuos_create); wall time from the first gpuos_submit to gpuos_wait(ALL)"}
+    except Exception as ex:  # reported, never fatal to the bench line
+        live = {"error": str(ex)[:200]}
+
     baselines = None
     if args.baselines and rank == 0:
         baselines = run_baselines(args, G, torch, stream, descs, n, dev)
@@ -354,6 +375,7 @@ def bench_gpu(args, rank, world, local):
         "hbm_gbs": achieved,
         "hbm_frac_of_nominal_8000": achieved / NOMINAL_HBM_GBS,
         "host_submit_us_per_op": submit_us,
+        "live_api": live,
         "gpu_span_ms_last_step": span_ns / 1e6,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": peak_kind, "traffic": profiled_traffic(args.config)},
