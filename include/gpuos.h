@@ -140,6 +140,7 @@ typedef struct gpuos_config {
 #define GPUOS_CFG_TRACE 2u        /* record a per-op event log (gpuos_trace_read) */
 #define GPUOS_CFG_NO_BULK 4u      /* op bodies read operands with plain loads only, no bulk-copy staging */
 #define GPUOS_CFG_NO_HANDOFF 8u   /* no chain hand-off: a claimed op always waits for its dependencies where it was claimed */
+#define GPUOS_CFG_NO_FUSION 16u   /* no fused pairs: every submitted op runs as its own entry */
 
 #define GPUOS_START_DRAIN 1u      /* the kernel exits once every op published before gpuos_start completed */
 

@@ -53,6 +53,12 @@ GPUOS_HD bool hdr_follow(u64 h) { return (h & HDR_FOLLOW) != 0; }
 constexpr u64 BIG_COUNT_MASK = (1ull << 24) - 1;
 constexpr u64 BIG_EXHAUSTED = 1ull << 23;  // count that exceeds every op's items
 
+// Internal micro-op (never accepted from callers): store the accumulator as an
+// output at in1. The runtime fuses two consecutive dependent scalar elementwise
+// ops A -> B into A's entry as progA, M_STORE1, progB (in1 = A's output, out =
+// B's output) and turns B into a NOP that depends on A.
+constexpr unsigned char M_STORE1 = 11;
+
 GPUOS_HD bool op_is_row(int op) {
   return op == GPUOS_OP_ROWSUM || op == GPUOS_OP_ROWMAX || op == GPUOS_OP_SOFTMAX ||
          op == GPUOS_OP_RMSNORM || op == GPUOS_OP_LAYERNORM || op == GPUOS_OP_ROTARY;

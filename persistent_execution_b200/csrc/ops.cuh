@@ -550,6 +550,95 @@ static __device__ __noinline__ void ew_stream(const RingEntry& E, u32 item, u32 
   __syncwarp();
 }
 
+// A fused pair (see M_STORE1): scalar micro-ops only, with one store of the
+// intermediate accumulator to in1. Both outputs are written, as two separate
+// ops would write them.
+__device__ __forceinline__ bool chain_has_store(const RingEntry& E) {
+  bool st = false;
+  for (int i = 0; i < E.nmicro; ++i) st |= E.micro[i] == M_STORE1;
+  return st;
+}
+__device__ __forceinline__ void chain8_store(const RingEntry& E, float (&a)[8], float (&mid)[8]) {
+  int k = 0;
+  const int nm = E.nmicro;
+  for (int i = 0; i < nm; ++i) {
+    const int m = E.micro[i];
+    if (m == GPUOS_M_AFFINE) {
+      const float s0 = E.s[k & 3], s1 = E.s[(k + 1) & 3];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a[j] = __fmaf_rn(s0, a[j], s1);
+      k += 2;
+    } else if (m == GPUOS_M_RELU) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a[j] = relu_f(a[j]);
+    } else if (m == GPUOS_M_SCALE) {
+      const float s0 = E.s[k & 3];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a[j] = __fmul_rn(a[j], s0);
+      k += 1;
+    } else if (m == GPUOS_M_ADDS) {
+      const float s0 = E.s[k & 3];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a[j] = __fadd_rn(a[j], s0);
+      k += 1;
+    } else if (m == M_STORE1) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) mid[j] = a[j];
+    }
+  }
+}
+
+// Body of a fused pair: one item of whole or ragged tiles, in0 read once,
+// the intermediate written to in1 and the result to out.
+template <int DT>
+static __device__ __noinline__ void ew_fused(const RingEntry& E, u32 item, u32 elem_chunk, const Cx cx) {
+  const long long n = E.rows * E.cols;
+  const long long e0 = (long long)item * elem_chunk;
+  const long long e1 = min(n, e0 + (long long)elem_chunk);
+  const long long n0 = E.in_n0;
+  const bool vec = n0 == n && al16(E.in0) && al16(E.in1) && al16(E.out);
+  const int lane = cx.lane, w = cx.warp, NW = cx.nwarps;
+  const long long full = (e1 - e0) / EW_TILE, tiles = (e1 - e0 + EW_TILE - 1) / EW_TILE;
+  long long t = w;
+  if (vec) {
+    for (; t + NW < full; t += 2ll * NW) {
+      float a[2][8], mid[2][8];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) tile_ld<DT>(E.in0, e0 + (t + (long long)u * NW) * EW_TILE, lane, a[u]);
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const long long t0 = e0 + (t + (long long)u * NW) * EW_TILE;
+        chain8_store(E, a[u], mid[u]);
+        tile_st<DT>(E.in1, t0, lane, mid[u]);
+        tile_st<DT>(E.out, t0, lane, a[u]);
+      }
+    }
+    for (; t < full; t += NW) {
+      const long long t0 = e0 + t * EW_TILE;
+      float a[8], mid[8];
+      tile_ld<DT>(E.in0, t0, lane, a);
+      chain8_store(E, a, mid);
+      tile_st<DT>(E.in1, t0, lane, mid);
+      tile_st<DT>(E.out, t0, lane, a);
+    }
+  }
+  const long long s0 = n0 < n ? (long long)umod(32, (u64)n0) : 32;
+  for (; t < tiles; t += NW) {
+    const long long t0 = e0 + t * EW_TILE;
+    float a[8], mid[8];
+    tile_gather<DT>(E.in0, t0, lane, n0, n, s0, e1, a);
+    chain8_store(E, a, mid);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const long long e = t0 + lane + 32 * k;
+      if (e < e1) {
+        st1<DT>(E.in1, e, mid[k]);
+        st1<DT>(E.out, e, a[k]);
+      }
+    }
+  }
+}
+
 __device__ __forceinline__ bool chain_calls(const RingEntry& E) {
   bool c = false;
   for (int i = 0; i < E.nmicro; ++i) c |= (E.micro[i] == GPUOS_M_GELU || E.micro[i] == GPUOS_M_SILU);
@@ -559,6 +648,10 @@ __device__ __forceinline__ bool chain_calls(const RingEntry& E) {
 template <int DT>
 __device__ void ew_item(const RingEntry& E, u32 item, u32 elem_chunk, const Cx& cx) {
   const long long n = E.rows * E.cols;
+  if (E.opcode == GPUOS_OP_EW_CHAIN && chain_has_store(E)) {
+    ew_fused<DT>(E, item, elem_chunk, cx);
+    return;
+  }
   // Bulk-copy staging pays off when the whole grid streams one large op from
   // HBM (an op of several items); a single-item op is latency-bound on one SM,
   // where the register path's loads arrive sooner.

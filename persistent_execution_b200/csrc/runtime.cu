@@ -153,6 +153,8 @@ struct gpuos {
   u64 cap = 0, mask = 0;
   u64 next_id = 0, published = 0, tail = 0, session_base = 0;
   u64 dma_upto = 0;               // ids below this were copied into the device ring by the copy engine
+  RingEntry last_e;               // entry of op next_id - 1 as written to the ring
+  bool last_fusable = false;      // that op may head a fused pair
   cudaEvent_t dma_ev = nullptr;   // the last such copy
   bool running = false;
   bool kernel_alive = false;  // false only if a kernel could not be confirmed stopped
@@ -398,6 +400,77 @@ gpuos_status wait_impl(gpuos* rt, u64 id, u64 timeout_ns) {
   }
 }
 
+// Fused pairs (NEXT step of the method: dynamic fusion of consecutive
+// elementwise ops, GPUOS page, "The Paper" and "What's New"; "Launch Overhead
+// and Fusion", "Fusion"). An fp32 single-item op whose program is scalar
+// micro-ops only (relu-affine or a chain of affine/scale/adds/relu) can head a
+// pair; the next op, if it is the same kind of op, reads the head's output as
+// its direct first operand over the same elements and depends on the head
+// alone, is folded into the head's entry while both are still unpublished.
+// The program becomes head, M_STORE1, tail with in1 = the head's output: both
+// outputs are written, bit-identical to running the two ops one after the
+// other (each micro-op rounds to fp32 either way). The tail becomes a NOP that
+// depends on the head, so completion order and dependants are unchanged.
+int scalar_program(const RingEntry& e, unsigned char* prog, int* nscal) {
+  if (e.opcode == GPUOS_OP_RELU_AFFINE) {
+    prog[0] = GPUOS_M_AFFINE;
+    prog[1] = GPUOS_M_RELU;
+    *nscal = 2;
+    return 2;
+  }
+  if (e.opcode != GPUOS_OP_EW_CHAIN) return -1;
+  int k = 0;
+  for (int i = 0; i < e.nmicro; ++i) {
+    const int m = e.micro[i];
+    if (m == GPUOS_M_AFFINE)
+      k += 2;
+    else if (m == GPUOS_M_SCALE || m == GPUOS_M_ADDS)
+      k += 1;
+    else if (m != GPUOS_M_RELU)
+      return -1;
+    prog[i] = (unsigned char)m;
+  }
+  *nscal = k;
+  return e.nmicro;
+}
+
+bool fusable(const RingEntry& e, bool single) {
+  unsigned char prog[8];
+  int ns = 0;
+  return single && e.dtype == GPUOS_F32 && e.in_n0 == e.rows * e.cols && scalar_program(e, prog, &ns) >= 0 &&
+         ns <= 4;
+}
+
+// Folds entry b (op id) into the previous entry a; true if fused.
+bool try_fuse(gpuos* rt, u64 id, RingEntry& a, const RingEntry& b) {
+  if ((rt->cfg.flags & GPUOS_CFG_NO_FUSION) || !rt->last_fusable || id == 0 || id - 1 < rt->published) return false;
+  if (b.in0 != a.out || b.rows * b.cols != a.rows * a.cols || b.in_n0 != a.rows * a.cols) return false;
+  if (!((b.dep0 == id && b.dep1 == 0) || (b.dep1 == id && b.dep0 == 0))) return false;  // depends on id - 1 alone
+  unsigned char pa[8], pb[8];
+  int ka = 0, kb = 0;
+  const int na = scalar_program(a, pa, &ka), nb = scalar_program(b, pb, &kb);
+  if (na < 0 || nb < 0 || ka + kb > 4 || na + 1 + nb > 8) return false;
+  RingEntry f = a;
+  f.opcode = GPUOS_OP_EW_CHAIN;
+  for (int i = 0; i < na; ++i) f.micro[i] = pa[i];
+  f.micro[na] = M_STORE1;
+  for (int i = 0; i < nb; ++i) f.micro[na + 1 + i] = pb[i];
+  for (int i = na + 1 + nb; i < 8; ++i) f.micro[i] = 0;
+  f.nmicro = (unsigned char)(na + 1 + nb);
+  for (int i = 0; i < kb; ++i) f.s[ka + i] = b.s[i];
+  f.in1 = a.out;
+  f.in_n1 = a.rows * a.cols;
+  f.out = b.out;
+  a = f;
+  return true;
+}
+
+void write_entry(gpuos* rt, u64 id, const RingEntry& e) {
+  __m128i* dst = reinterpret_cast<__m128i*>(&rt->hring[id & rt->mask]);
+  const __m128i* src = reinterpret_cast<const __m128i*>(&e);
+  for (int j = 0; j < 8; ++j) _mm_stream_si128(dst + j, _mm_load_si128(src + j));
+}
+
 gpuos_status submit_one(gpuos* rt, const gpuos_desc* d, u64 dep_base, u64 first_id, u64* id_out, bool raw) {
   if (rt->sticky != GPUOS_OK) return rt->sticky;
   if (!raw) {
@@ -464,10 +537,24 @@ gpuos_status submit_one(gpuos* rt, const gpuos_desc* d, u64 dep_base, u64 first_
     rt->big_ids.push_back(id);
   }
   e.hdr = hdr_make(id, follow, items);
+  bool fused = false;
+  if (single && try_fuse(rt, id, rt->last_e, e)) {
+    // the previous entry now computes both ops; this one only completes after it
+    write_entry(rt, id - 1, rt->last_e);
+    RingEntry nop;
+    std::memset(&nop, 0, sizeof(nop));
+    nop.opcode = GPUOS_OP_NOP;
+    nop.rows = nop.cols = 1;
+    nop.in_n0 = nop.in_n1 = 1;
+    nop.dep0 = id;  // id - 1, encoded as id + 1 of it
+    nop.hdr = hdr_make(id, follow, 1);
+    e = nop;
+    fused = true;
+  }
   // write the 128-byte entry into the write-combined ring
-  __m128i* dst = reinterpret_cast<__m128i*>(&rt->hring[id & rt->mask]);
-  const __m128i* src = reinterpret_cast<const __m128i*>(&e);
-  for (int j = 0; j < 8; ++j) _mm_stream_si128(dst + j, _mm_load_si128(src + j));
+  write_entry(rt, id, e);
+  rt->last_e = e;
+  rt->last_fusable = !fused && fusable(e, single);
   rt->prev_chain_start = follow ? rt->prev_chain_start : id;
   rt->prev_single = single;
   rt->next_id = id + 1;

@@ -33,6 +33,7 @@ CFG_NO_AUTOSTART = 1
 CFG_TRACE = 2
 CFG_NO_BULK = 4
 CFG_NO_HANDOFF = 8
+CFG_NO_FUSION = 16
 START_DRAIN = 1
 
 # numpy view of gpuos_desc (128 bytes), for building many descriptors at once

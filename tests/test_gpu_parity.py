@@ -168,6 +168,20 @@ def test_dependent_elementwise_chains_bit_exact(dtype, n):
     assert P.bit_exact(w, a32, a16, r32, r16) == []
 
 
+@pytest.mark.parametrize("config", [1, 2, 5])
+def test_fused_pairs_match_unfused(config):
+    # consecutive dependent scalar elementwise ops are fused into pairs at
+    # submit; outputs must be bit-identical with fusion off, and match the oracle
+    w = W.make(config, small=True)
+    a32, a16, _, _ = U.run_persistent(w)
+    assert not P.check_ops(w, a32, a16, idx=P.teacher_forcible(w) if config == 5 else None)
+    b32, b16, _, _ = U.run_persistent(w, cfg=dict(flags=G.CFG_NO_FUSION))
+    assert np.array_equal(a32.view(np.uint32), b32.view(np.uint32)) and np.array_equal(a16, b16)
+    if config == 1:
+        r32, r16 = oracle.run(w)
+        assert P.bit_exact(w, a32, a16, r32, r16) == []
+
+
 @pytest.mark.parametrize("mode", ["drain", "live"])
 def test_chain_handoff_interleaved_streams(mode):
     # config 4's request chains are interleaved, so a claimed op's predecessor
