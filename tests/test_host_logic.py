@@ -95,3 +95,21 @@ def test_generators_are_seeded_and_structured():
     w4 = W.make(4, small=True)
     s = w4.meta["streams"]
     assert (w4.ops["dep"][s:, 0] == np.arange(w4.n_ops - s)).all()
+
+
+def test_algorithmic_bytes_per_op_kind():
+    # each distinct operand element read once (a broadcast operand counts its
+    # own elements), each output written once, weights once per op
+    b = W._Builder("bytes", 0)
+    f = b.alloc_input(0, np.zeros(4096, np.float32))
+    h = b.alloc_input(1, np.zeros(4096, np.uint16))
+    o32, o16 = b.alloc_output(0, 4096), b.alloc_output(1, 4096)
+    b.add_op("rowsum", 0, [f], o32, 8, 100, in_n=(800, 0))
+    b.add_op("softmax", 1, [h], o16, 4, 64, in_n=(256, 0))
+    b.add_op("rmsnorm", 1, [h, h], o16, 2, 128, in_n=(256, 128), s=(1e-6, 0, 0, 0))
+    b.add_op("layernorm", 0, [f, f, f], o32, 3, 32, in_n=(96, 32), s=(1e-5, 0, 0, 0))
+    b.add_op("add", 0, [f, f], o32, 1, 1000, in_n=(7, 1000))
+    b.add_op("rotary", 1, [h], o16, 16, 128, in_n=(2048, 0), s=(10000.0, 0, 0, 0), pos=3)
+    by = measure.op_bytes(b.finish()).tolist()
+    assert by == [8 * 100 * 4 + 8 * 4, 2 * 256 * 2, (2 * 256 + 128) * 2, (2 * 96 + 2 * 32) * 4,
+                  (7 + 1000 + 1000) * 4, 2 * 2048 * 2]
